@@ -1,0 +1,153 @@
+"""Python access to the fp64 CPU oracle (``mate_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
+baseline use this package; the product path never imports it.
+
+The wrapper marshals arrays only: every step of the computation runs in the
+C file. Inputs are upcast to float64 exactly (bf16 and fp32 values are
+representable in fp64), so the oracle sees the very values the GPU sees.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "mate_oracle.c")
+BUILD_DIR = os.path.join(_HERE, "_build")
+DEFAULT_LIB = os.path.join(BUILD_DIR, "liboracle.so")
+
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_intp = ctypes.POINTER(ctypes.c_int)
+
+
+def build(source: str = SOURCE, out: str = DEFAULT_LIB, extra: Sequence[str] = ()) -> str:
+    """Compile the oracle into a shared library (gcc, -O2, OpenMP, IEEE fp64)."""
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    if (os.path.exists(out) and not extra and source == SOURCE
+            and os.path.getmtime(out) >= os.path.getmtime(source)):
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+           "-ffp-contract=off", *extra, source, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # torch tensor: exact upcast, then numpy
+        a = a.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+class Oracle:
+    """ctypes handle on one build of the oracle library."""
+
+    def __init__(self, lib_path: Optional[str] = None):
+        path = lib_path or build()
+        self.path = path
+        self.lib = ctypes.CDLL(path)
+        L = self.lib
+        L.oracle_unroll.argtypes = [ctypes.c_int] * 3 + [_intp, _i32p]
+        L.oracle_rms_sequence.argtypes = [ctypes.c_int] * 5 + [_i32p]
+        L.oracle_avg_pool.argtypes = [_f64p] + [ctypes.c_int] * 7 + [_f64p]
+        L.oracle_ssd_scan.argtypes = [ctypes.c_int64] + [ctypes.c_int] * 4 + [_f64p] * 6 + [_f64p]
+        L.oracle_bissd.argtypes = [ctypes.c_int] * 8 + [_f64p] * 6 + [ctypes.c_int, _intp, _f64p]
+        L.oracle_tesa_window_ids.argtypes = [ctypes.c_int] * 5 + [_intp, _i32p]
+        L.oracle_tesa.argtypes = [ctypes.c_int] * 6 + [_f64p] * 3 + [ctypes.c_int] * 2 + [_intp, _f64p]
+        for f in ("oracle_unroll", "oracle_rms_sequence", "oracle_avg_pool", "oracle_ssd_scan",
+                  "oracle_bissd", "oracle_tesa_window_ids", "oracle_tesa"):
+            getattr(L, f).restype = ctypes.c_int
+
+    # ---- Rotary Major Scan -------------------------------------------------
+    def unroll(self, T: int, H: int, W: int, priority: Sequence[int]) -> np.ndarray:
+        seq = np.empty(T * H * W, dtype=np.int32)
+        pr = (ctypes.c_int * 3)(*priority)
+        rc = self.lib.oracle_unroll(T, H, W, pr, _ptr(seq, _i32p))
+        if rc:
+            raise ValueError(f"oracle_unroll rc={rc}")
+        return seq
+
+    def rms_sequence(self, T: int, H: int, W: int, mode: int, flip: bool = False) -> np.ndarray:
+        seq = np.empty(T * H * W, dtype=np.int32)
+        rc = self.lib.oracle_rms_sequence(T, H, W, mode, int(bool(flip)), _ptr(seq, _i32p))
+        if rc:
+            raise ValueError(f"oracle_rms_sequence rc={rc}")
+        return seq
+
+    def avg_pool(self, grid, pool) -> np.ndarray:
+        g = _f64(grid)
+        T, H, W = g.shape[:3]
+        ch = int(np.prod(g.shape[3:])) if g.ndim > 3 else 1
+        pt, ph, pw = pool
+        out = np.empty((T // pt, H // ph, W // pw) + g.shape[3:], dtype=np.float64)
+        rc = self.lib.oracle_avg_pool(_ptr(g, _f64p), T, H, W, ch, pt, ph, pw, _ptr(out, _f64p))
+        if rc:
+            raise ValueError(f"oracle_avg_pool rc={rc}")
+        return out
+
+    # ---- SSD ---------------------------------------------------------------
+    def ssd_scan(self, x, dt, A, B, C, D) -> np.ndarray:
+        """One-direction scan of an explicit sequence. x: (L, nh, P); dt: (L, nh);
+        B, C: (L, G, Ns); A, D: (nh,)."""
+        x, dt, A, B, C, D = map(_f64, (x, dt, A, B, C, D))
+        L, nh, P = x.shape
+        G, Ns = B.shape[1:]
+        y = np.empty_like(x)
+        rc = self.lib.oracle_ssd_scan(L, nh, P, Ns, G, _ptr(x, _f64p), _ptr(dt, _f64p), _ptr(A, _f64p),
+                                      _ptr(B, _f64p), _ptr(C, _f64p), _ptr(D, _f64p), _ptr(y, _f64p))
+        if rc:
+            raise ValueError(f"oracle_ssd_scan rc={rc}")
+        return y
+
+    def bissd(self, x, dt, A, B, C, D, mode: int, pool=None) -> np.ndarray:
+        """x: (batch, T, H, W, nh, P); dt: (batch, T, H, W, nh); B, C: (batch, T, H, W, G, Ns)."""
+        x, dt, A, B, C, D = map(_f64, (x, dt, A, B, C, D))
+        b, T, H, W, nh, P = x.shape
+        G, Ns = B.shape[4:]
+        out = np.empty_like(x)
+        pl = (ctypes.c_int * 3)(*(pool if pool else (0, 0, 0)))
+        rc = self.lib.oracle_bissd(b, T, H, W, nh, P, Ns, G, _ptr(x, _f64p), _ptr(dt, _f64p), _ptr(A, _f64p),
+                                   _ptr(B, _f64p), _ptr(C, _f64p), _ptr(D, _f64p), mode, pl, _ptr(out, _f64p))
+        if rc:
+            raise ValueError(f"oracle_bissd rc={rc}")
+        return out
+
+    # ---- TESA --------------------------------------------------------------
+    def tesa_window_ids(self, T: int, H: int, W: int, Tw: int, Sw: int, shift) -> np.ndarray:
+        win = np.empty(T * H * W, dtype=np.int32)
+        sh = (ctypes.c_int * 3)(*shift)
+        rc = self.lib.oracle_tesa_window_ids(T, H, W, Tw, Sw, sh, _ptr(win, _i32p))
+        if rc < 0:
+            raise ValueError(f"oracle_tesa_window_ids rc={rc}")
+        return win
+
+    def tesa(self, q, k, v, Tw: int, Sw: int, shift) -> np.ndarray:
+        q, k, v = map(_f64, (q, k, v))
+        b, T, H, W, nh, d = q.shape
+        out = np.empty_like(q)
+        sh = (ctypes.c_int * 3)(*shift)
+        rc = self.lib.oracle_tesa(b, T, H, W, nh, d, _ptr(q, _f64p), _ptr(k, _f64p), _ptr(v, _f64p),
+                                  Tw, Sw, sh, _ptr(out, _f64p))
+        if rc < 0:
+            raise ValueError(f"oracle_tesa rc={rc}")
+        return out
+
+
+_default: Optional[Oracle] = None
+
+
+def get() -> Oracle:
+    """The oracle built from the committed source (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

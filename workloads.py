@@ -1,0 +1,136 @@
+"""Seeded synthetic workloads for the MATE token-mix core.
+
+This module only describes shapes and draws random inputs. It holds none of
+the method's arithmetic, so both the CUDA path (through its tests and the
+bench) and the CPU oracle can be fed from it without sharing any code.
+
+Shapes follow the five video-latent grids the token mix is measured on
+(a tiny fp32 case and 256p/512p/768p grids of 17 s to 68 s). The pages give
+no latent grid sizes, so these grids stand in for the pages' workloads; the
+layer widths come from the LinGen paper review (xllm-io), "5.1 实验设置":
+20 heads and embedding width 2560, with the Mamba2 head dimension 64 stated
+under "MA-Branch", item 1.
+
+Distributions (drawn on the host; the SSD inputs from a ``torch.Generator``
+seeded with ``seed`` in the order x, dt_raw, A_raw, B, C, D, the attention
+inputs q, k, v from a second generator seeded with ``seed + 1``, so that
+either set can be drawn without the other):
+    x ~ N(0, 1)
+    dt = softplus(N(0, 1) - 4)
+    A = -exp(U(0, ln 16))          (long-memory variant: divided by 256)
+    B, C ~ N(0, 1) / sqrt(d_state)
+    D ~ N(0, 1)
+    q, k, v ~ N(0, 1)
+Tensors the config marks bf16 (x, B, C, q, k, v) are cast to bf16 after the
+draw; dt, A and D stay fp32.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+from typing import Dict, Optional, Tuple
+
+import torch
+
+# scan-mode codes shared by every layer of the stack
+SR, SC, TR, TC = 0, 1, 2, 3
+MODE_NAMES = {SR: "spatial-row", SC: "spatial-column", TR: "temporal-row", TC: "temporal-column"}
+
+
+@dataclass(frozen=True)
+class Config:
+    name: str
+    batch: int
+    T: int
+    H: int
+    W: int
+    # SSD (MA-branch)
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    chunk: int
+    dtype: str                      # "f32" or "bf16" for x, B, C, q, k, v, out
+    modes: Tuple[int, ...]          # RMS modes exercised by this config
+    review: Optional[Tuple[int, int, int]]   # pooling kernel (pt, ph, pw) or None
+    # TESA (TE-branch)
+    attn_heads: int
+    attn_dim: int
+    Tw: int
+    Sw: int
+    shift: Tuple[int, int, int]
+    variant: str = "default"        # "default" or "long_memory"
+
+    @property
+    def N(self) -> int:
+        return self.T * self.H * self.W
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.N
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def with_(self, **kw) -> "Config":
+        return replace(self, **kw)
+
+
+CONFIGS: Dict[str, Config] = {
+    "tiny": Config("tiny", 1, 4, 8, 8, 2, 16, 16, 1, 32, "f32", (SR, SC, TR, TC), (2, 4, 4),
+                   2, 16, 2, 4, (1, 2, 2)),
+    "256p-17s": Config("256p-17s", 1, 32, 16, 16, 80, 64, 64, 1, 256, "bf16", (SR,), None,
+                       20, 128, 2, 8, (0, 0, 0)),
+    "512p-17s": Config("512p-17s", 1, 32, 32, 32, 80, 64, 64, 1, 256, "bf16", (SR, SC, TR, TC),
+                       (4, 8, 8), 20, 128, 2, 8, (1, 4, 4)),
+    "512p-68s": Config("512p-68s", 1, 128, 32, 32, 80, 64, 64, 1, 256, "bf16", (TC,), (8, 8, 8),
+                       20, 128, 2, 8, (1, 4, 4)),
+    "768p-17s": Config("768p-17s", 2, 32, 48, 48, 80, 64, 64, 1, 256, "bf16", (SR, SC, TR, TC), None,
+                       20, 128, 2, 8, (0, 0, 0)),
+}
+
+# the grid the headline throughput is quoted on (131,072 tokens)
+HEADLINE = "512p-68s"
+
+
+def sweep_configs():
+    """N from 8k to 131k tokens at H=W=32 with the 131k grid's other settings."""
+    base = CONFIGS[HEADLINE]
+    return [base.with_(name=f"sweep-T{t}", T=t) for t in (8, 16, 32, 64, 128)]
+
+
+def generate(cfg: Config, seed: int = 0, parts: Tuple[str, ...] = ("ssd", "attn")) -> Dict[str, torch.Tensor]:
+    """Draw one batch of inputs on the host.
+
+    The draw order within each stream is fixed, and the two streams are
+    independent, so a config's SSD inputs do not depend on whether the
+    attention inputs are drawn too.
+    Returns CPU tensors in grid order (batch, T, H, W, ...).
+    """
+    g = torch.Generator().manual_seed(seed)
+    b, T, H, W = cfg.batch, cfg.T, cfg.H, cfg.W
+    out: Dict[str, torch.Tensor] = {}
+    dt_ = cfg.torch_dtype
+    if "ssd" in parts:
+        x = torch.randn(b, T, H, W, cfg.nheads, cfg.headdim, generator=g)
+        dt_raw = torch.randn(b, T, H, W, cfg.nheads, generator=g)
+        a_raw = torch.rand(cfg.nheads, generator=g)
+        Bm = torch.randn(b, T, H, W, cfg.ngroups, cfg.dstate, generator=g) / math.sqrt(cfg.dstate)
+        Cm = torch.randn(b, T, H, W, cfg.ngroups, cfg.dstate, generator=g) / math.sqrt(cfg.dstate)
+        D = torch.randn(cfg.nheads, generator=g)
+        dt = torch.nn.functional.softplus(dt_raw - 4.0)
+        A = -torch.exp(a_raw * math.log(16.0))
+        if cfg.variant == "long_memory":
+            A = A / 256.0
+        out.update(x=x.to(dt_), dt=dt.float().contiguous(), A=A.float(), B=Bm.to(dt_), C=Cm.to(dt_),
+                   D=D.float())
+    if "attn" in parts:
+        ga = torch.Generator().manual_seed(seed + 1)
+        shape = (b, T, H, W, cfg.attn_heads, cfg.attn_dim)
+        q = torch.randn(*shape, generator=ga)
+        k = torch.randn(*shape, generator=ga)
+        v = torch.randn(*shape, generator=ga)
+        out.update(q=q.to(dt_), k=k.to(dt_), v=v.to(dt_))
+    return out
+
