@@ -1,0 +1,420 @@
+"""Throughput of the MATE token mix on B200: one step = review pooling and
+prefix scan, the bidirectional SSD scan and TESA over one batch of a
+synthetic latent grid.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl mate|reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun, one rank per GPU) every
+rank processes its own batch element drawn with its own seed: the path has
+no exchange step, so this is weak scaling with no collective on the data
+path; the NCCL group only carries the barrier and the max-over-ranks time.
+
+--impl reference times the fp64 CPU oracle (the only other code this script
+may run) on the same workload, one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes per token of each kernel (one read of what the step
+# must read, one write of what it must write)
+# ---------------------------------------------------------------------------
+def elem_bytes(cfg):
+    return 4 if cfg.dtype == "f32" else 2
+
+
+def algorithmic_bytes(cfg):
+    e = elem_bytes(cfg)
+    x = cfg.nheads * cfg.headdim * e
+    dt = cfg.nheads * 4
+    bc = cfg.ngroups * cfg.dstate * e
+    per_tok = {
+        "review_pool": (x + dt + bc) if cfg.review else 0,   # x, dt, B (C is never needed)
+        "chunk_state": x + dt + bc,                          # x, dt, B
+        "chunk_out": 2 * x + dt + 2 * bc,                    # x, dt, B, C in; y out
+        "tesa": 4 * cfg.attn_heads * cfg.attn_dim * e,       # q, k, v in; out
+    }
+    per_tok["bissd"] = 2 * x + dt + 2 * bc                   # the MA-branch as one op
+    return per_tok
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid):
+        self.uuid = device_uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+def oracle_sample(cfg, threads=None):
+    """Time the fp64 oracle on a head subset of the full grid and scale to the
+    whole workload (heads are independent, so cost is linear in heads).
+    Returns (Mtokens/s, cores, description)."""
+    import oracle
+
+    threads = threads or min(os.cpu_count() or 1, 16)
+    os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+    o = oracle.get()
+    ssd_heads = min(cfg.nheads, threads)
+    attn_heads = min(cfg.attn_heads, 2)
+    inp = workloads.generate(cfg.with_(batch=1), seed=0)
+    x = inp["x"][..., :ssd_heads, :]
+    dt = inp["dt"][..., :ssd_heads]
+    A = inp["A"][:ssd_heads]
+    D = inp["D"][:ssd_heads]
+    mode = cfg.modes[0]
+    t0 = time.perf_counter()
+    o.bissd(x, dt, A, inp["B"], inp["C"], D, mode, cfg.review)
+    t_ssd = time.perf_counter() - t0
+    q, k, v = (inp[n][..., :attn_heads, :] for n in ("q", "k", "v"))
+    t0 = time.perf_counter()
+    o.tesa(q, k, v, cfg.Tw, cfg.Sw, cfg.shift)
+    t_attn = time.perf_counter() - t0
+    t_full = t_ssd * cfg.nheads / ssd_heads + t_attn * cfg.attn_heads / attn_heads
+    desc = (f"{cfg.name} grid {cfg.T}x{cfg.H}x{cfg.W}, 1 batch element: bi-SSD on {ssd_heads}/{cfg.nheads} heads "
+            f"({t_ssd:.2f} s), TESA on {attn_heads}/{cfg.attn_heads} heads ({t_attn:.2f} s), "
+            f"scaled by head count to the full step")
+    return cfg.N / t_full / 1e6, threads, desc
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_mate(args, cfg, rank, world, dist):
+    import ctypes
+
+    import torch
+
+    import linear_complexity_video_b200 as mate
+    from linear_complexity_video_b200 import _lib, api
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    L = mate.load()
+    stream = torch.cuda.current_stream()
+    mode = cfg.modes[0]
+
+    host = workloads.generate(cfg, seed=rank)
+    d = {k: v.to(dev) for k, v in host.items()}
+    out_ssd = torch.empty_like(d["x"])
+    out_att = torch.empty_like(d["q"])
+    ws = api.bissd_workspace(d["x"], d["B"], cfg.review, cfg.chunk)
+    sdims = api.ssd_dims(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, cfg.ngroups, cfg.chunk, cfg.torch_dtype)
+    adims = api.attn_dims(cfg.batch, cfg.attn_heads, cfg.attn_dim, cfg.torch_dtype)
+
+    def step(src, o_ssd, o_att, workspace):
+        api.mate_bissd_fwd(src["x"], src["dt"], src["A"], src["B"], src["C"], src["D"], cfg.T, cfg.H, cfg.W, mode,
+                           cfg.review, o_ssd, sdims, workspace, stream)
+        api.tesa_fwd(src["q"], src["k"], src["v"], cfg.T, cfg.H, cfg.W, cfg.Tw, cfg.Sw, cfg.shift, o_att, adims,
+                     stream)
+
+    # phase events recorded through the library's enqueue-time hook
+    marks = []
+
+    def hook(phase, is_end, strm, user):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        marks.append((phase, is_end, ev))
+
+    hook_c = _lib.PHASE_HOOK(hook)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(d, out_ssd, out_att, ws)
+    torch.cuda.synchronize()
+    rc = mate.mate_last_error()
+    if rc != 0:
+        raise RuntimeError(f"device error word {rc}")
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}") if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    launches0 = L.mate_kernel_launches()
+    L.mate_set_phase_hook(hook_c, None)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(d, out_ssd, out_att, ws)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    L.mate_set_phase_hook(_lib.PHASE_HOOK(), None)
+    launches = L.mate_kernel_launches() - launches0
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_total = ev0.elapsed_time(ev1)
+    t_local = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    ms_total = float(t_local.item())
+    ms_step = ms_total / args.steps
+
+    # per-phase average duration on this rank
+    phase_ms = {}
+    open_ev = {}
+    for phase, is_end, ev in marks:
+        if not is_end:
+            open_ev[phase] = ev
+        else:
+            phase_ms.setdefault(_lib.PHASES[phase], []).append(open_ev.pop(phase).elapsed_time(ev))
+    phase_avg = {k: sum(v) / len(v) for k, v in phase_ms.items()}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pinned = {k: v.pin_memory() for k, v in host.items()}
+        h_ssd = torch.empty(out_ssd.shape, dtype=out_ssd.dtype).pin_memory()
+        h_att = torch.empty(out_att.shape, dtype=out_att.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+        d2h = h_ssd.numel() * h_ssd.element_size() + h_att.numel() * h_att.element_size()
+
+        def e2e_step():
+            for k_, v_ in pinned.items():
+                d[k_].copy_(v_, non_blocking=True)
+            step(d, out_ssd, out_att, ws)
+            h_ssd.copy_(out_ssd, non_blocking=True)
+            h_att.copy_(out_att, non_blocking=True)
+
+        for _ in range(min(args.warmup, 2)):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        k_e2e = max(1, min(args.steps, args.e2e_steps))
+        e0.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / k_e2e], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": cfg.tokens * world / (float(te.item()) / 1e3) / 1e6, "unit": "Mtokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e}
+
+    result = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        per_tok = algorithmic_bytes(cfg)
+        # dominant kernel by time
+        dom = max(phase_avg, key=lambda k: phase_avg[k])
+        dom_bytes = per_tok.get(dom, 0) * cfg.tokens
+        achieved = dom_bytes / (phase_avg[dom] / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        value = cfg.tokens * world / (ms_step / 1e3) / 1e6
+        traffic = load_traffic(dom, cfg)
+        result = {
+            "metric": "MATE token-mix Mtokens/s on 1 B200 (bi-SSD+TESA)",
+            "value": value,
+            "unit": "Mtokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded, per rank)",
+            "config": {"workload": f"{cfg.name}: grid T={cfg.T} H={cfg.H} W={cfg.W} x batch {cfg.batch}, "
+                                   f"SSD {cfg.nheads}x{cfg.headdim} d_state {cfg.dstate} chunk {cfg.chunk}, "
+                                   f"scan {workloads.MODE_NAMES[mode]}, review pool {cfg.review}, "
+                                   f"TESA {cfg.attn_heads}x{cfg.attn_dim} window {cfg.Tw}x{cfg.Sw}x{cfg.Sw} "
+                                   f"shift {cfg.shift}",
+                       "tokens_per_rank": cfg.tokens, "global_tokens": cfg.tokens * world,
+                       "parallelism": f"dp{world} (independent grids)",
+                       "l2": f"inputs larger than L2 ({cfg.tokens * per_tok['bissd'] / 1e9:.2f} GB per bi-SSD pass "
+                             f"> {L2_BYTES / 1e6:.0f} MB); no flush"},
+            "phase_ms": {k: round(v, 4) for k, v in phase_avg.items()},
+            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_src},
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "e2e": e2e,
+        }
+    return result
+
+
+def load_traffic(kernel, cfg):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if one
+    matches the current build and workload; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = t.get(kernel)
+    if not ent or ent.get("workload") != cfg.name:
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def run_reference(args, cfg):
+    """The oracle, timed on the host cores, one bounded sample per step."""
+    vals = []
+    cores = None
+    desc = ""
+    for _ in range(args.warmup_ref):
+        oracle_sample(cfg)
+    for _ in range(args.steps_ref):
+        v, cores, desc = oracle_sample(cfg)
+        vals.append(v)
+    value = statistics.median(vals)
+    return {
+        "impl": "reference",
+        "metric": "MATE token-mix Mtokens/s on 1 B200 (bi-SSD+TESA)",
+        "value": value,
+        "unit": "Mtokens/s",
+        "n_gpus": 1,
+        "steps": len(vals),
+        "warmup": args.warmup_ref,
+        "ms_per_step": cfg.tokens / (value * 1e6) * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"{cfg.name}: grid T={cfg.T} H={cfg.H} W={cfg.W} x batch {cfg.batch}"},
+        "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=workloads.HEADLINE, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", default="mate", choices=["mate", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--steps-ref", type=int, default=1)
+    ap.add_argument("--warmup-ref", type=int, default=0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = workloads.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, cfg)), flush=True)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        res = run_mate(args, cfg, rank, world, dist)
+        if rank == 0:
+            if not args.no_cpu_baseline and world == 1:
+                v, cores, desc = oracle_sample(cfg)
+                res["cpu_baseline"] = {"value": v, "unit": "Mtokens/s", "cores": cores, "kind": "oracle",
+                                       "sample": desc}
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,219 @@
+/*
+ * mate.h - C ABI of the MATE token-mix library (libmate.so) for NVIDIA B200
+ * (sm_100a).
+ *
+ * The library computes the token-mixing core of LinGen's MATE block, the
+ * linear-complexity block that replaces DiT self-attention:
+ *   - the MA-branch: a bidirectional Mamba2 (SSD) selective scan over the
+ *     T x H x W latent token grid, unrolled in one of the four Rotary Major
+ *     Scan orders, optionally preceded by review tokens;
+ *   - the TE-branch: TEmporal Swin Attention (TESA), softmax attention inside
+ *     fixed Tw x Sw x Sw windows whose placement is shifted on alternate
+ *     layers.
+ * Sources: "LinGen: Towards High-Resolution Minute-Length Text-to-Video
+ * Generation with Linear Computational Complexity" (xllm-io paper review),
+ * section 三 "技术架构", MA-Branch items 1-3 and TE-Branch; the QbitAI news
+ * article on LinGen, method section.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The
+ *     library allocates no device memory and keeps no state between calls,
+ *     apart from one device-side error word (see mate_last_error).
+ *   - Tensors are dense and contiguous in grid order: for a batch element,
+ *     token (t, h, w) sits at grid offset (t*H + h)*W + w, W fastest.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Work is enqueued on it; calls return before it finishes.
+ *   - Inputs are never written. Outputs must not overlap any input.
+ *   - Return value: MATE_OK, or a negative MATE_ERR_* code. Argument errors
+ *     are detected on the host before anything is enqueued; nothing is
+ *     written then.
+ */
+#ifndef MATE_H
+#define MATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define MATE_OK 0
+#define MATE_ERR_INVALID_ARG (-1) /* null or misaligned pointer, bad size, overlap  */
+#define MATE_ERR_UNSUPPORTED (-2) /* dims or dtype outside the compiled set          */
+#define MATE_ERR_CUDA (-3)        /* a CUDA launch or runtime call failed            */
+#define MATE_ERR_TIMEOUT (-4)     /* a bounded device-side wait gave up              */
+#define MATE_ERR_WORKSPACE (-5)   /* workspace missing, too small or misaligned      */
+
+/* ---- element types ------------------------------------------------------ */
+#define MATE_F32 0  /* x, B, C, q, k, v, out stored as IEEE fp32 */
+#define MATE_BF16 1 /* x, B, C, q, k, v, out stored as bf16; fp32 accumulation */
+
+/* ---- Rotary Major Scan orders (paper review, MA-Branch item 2) ----------
+ * Scan position n of a T x H x W grid maps to these grid coordinates:
+ *   SR spatial-row:     n = (t*H + h)*W + w      (W fastest, then H, then T)
+ *   SC spatial-column:  n = (t*W + w)*H + h      (H fastest, then W, then T)
+ *   TR temporal-row:    n = (h*W + w)*T + t      (T fastest, then W, then H)
+ *   TC temporal-column: n = (w*H + h)*T + t      (T fastest, then H, then W)
+ * The QbitAI article gives W, H, T the first, second and third priority in
+ * its example and obtains the other scans by exchanging priorities; "row"
+ * puts W before H, "temporal" puts T first. The flipped scan visits
+ * position N-1-n at step n (the review prints this as T*H*W - n with n
+ * counted from 1). */
+#define MATE_SCAN_SR 0
+#define MATE_SCAN_SC 1
+#define MATE_SCAN_TR 2
+#define MATE_SCAN_TC 3
+
+/* directions of the bidirectional scan (test and diagnosis aid) */
+#define MATE_DIR_FWD 1 /* the scan in RMS order only          */
+#define MATE_DIR_BWD 2 /* the flipped scan only, flipped back */
+#define MATE_DIR_BI 3  /* their sum (the MA-branch output)    */
+
+typedef struct {
+    int batch;      /* batch elements, >= 1                                  */
+    int nheads;     /* SSD heads nh                                          */
+    int headdim;    /* head dimension P                                      */
+    int dstate;     /* state size Ns (d_state)                               */
+    int ngroups;    /* B/C groups G; head h reads group h / (nh / G)         */
+    int chunk;      /* scan chunk length Q, a tiling choice: outputs do not  */
+                    /* depend on it beyond rounding                          */
+    int dtype;      /* MATE_F32 or MATE_BF16                                 */
+    int directions; /* MATE_DIR_*; 0 means MATE_DIR_BI                       */
+} mate_ssd_dims;
+
+typedef struct {
+    int batch;   /* batch elements, >= 1   */
+    int nheads;  /* attention heads        */
+    int headdim; /* head dimension d       */
+    int dtype;   /* MATE_F32 or MATE_BF16  */
+} mate_attn_dims;
+
+/*
+ * Workspace bytes mate_bissd_fwd needs for these dims (0 on bad arguments,
+ * which mate_bissd_fwd then reports). The workspace holds per-chunk scan
+ * states, chunk decays and, with review tokens, the pooled grid and the
+ * state the review prefix leaves behind. Its contents on entry do not
+ * matter.
+ */
+size_t mate_bissd_workspace_bytes(int T, int H, int W, const int review_pool[3], const mate_ssd_dims *d);
+
+/*
+ * MA-branch token mix: bidirectional Mamba2 / SSD scan in Rotary Major Scan
+ * order with optional review tokens (paper review, MA-Branch items 1-3).
+ *
+ * For each batch element and head h, let X be the grid unrolled in scan
+ * order `scan_mode` (N = T*H*W tokens). With state s (headdim x dstate,
+ * zero at the start of every scanned sequence) the scan computes
+ *     s_n = exp(dt_n * A[h]) * s_{n-1} + dt_n * x_n B_n^T
+ *     y_n = s_n C_n + D[h] * x_n
+ * once over [prefix, X] and once over [prefix, flip(X)]. The outputs at
+ * prefix positions are dropped, the second result is flipped back, and the
+ * two are added: out = y_forward + y_flipped (so D*x enters twice).
+ *
+ * Review tokens (review_pool = {pt, ph, pw}, all > 0 and dividing T, H, W):
+ * x, dt and B are average-pooled over non-overlapping pt x ph x pw boxes,
+ * the pooled grid is unrolled in the same scan order into R, and the prefix
+ * is [R, flip(R)] (2*T*H*W/(pt*ph*pw) tokens). That prefix reads the same
+ * forwards and backwards, so it precedes both scans unchanged. Outputs at
+ * prefix positions are dropped, so pooled C would never be used and is not
+ * computed. review_pool NULL or {0, 0, 0}: no prefix.
+ *
+ * Layouts (contiguous, grid order):
+ *   x, out : (batch, T, H, W, nheads, headdim)   dtype
+ *   dt     : (batch, T, H, W, nheads)            fp32, > 0 expected
+ *   A, D   : (nheads)                            fp32 (A < 0 expected)
+ *   B, C   : (batch, T, H, W, ngroups, dstate)   dtype
+ * x, B, C and out must be 16-byte aligned; dt, A, D 4-byte aligned.
+ * workspace: >= mate_bissd_workspace_bytes(...) bytes of device memory,
+ *   256-byte aligned, used only by the work this call enqueues.
+ * Supported: headdim and dstate in {16, 32, 64}, chunk in [1, 256],
+ *   nheads % ngroups == 0, T*H*W < 2^31.
+ * Returns MATE_OK, MATE_ERR_INVALID_ARG, MATE_ERR_UNSUPPORTED,
+ *   MATE_ERR_WORKSPACE or MATE_ERR_CUDA.
+ */
+int mate_bissd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                   const float *D, int T, int H, int W, int scan_mode, const int review_pool[3],
+                   void *out, const mate_ssd_dims *d, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * TE-branch: TEmporal Swin Attention (paper review, TE-Branch; the superapi
+ * product page, "Technical Principles": windows shift between layers).
+ *
+ * The grid is cut into windows of Tw x Sw x Sw tokens. Along each axis the
+ * window boundaries sit at the coordinates congruent to that axis' shift
+ * modulo the window size (shift = {st, sh, sw}, 0 <= st < Tw,
+ * 0 <= sh, sw < Sw), so with a non-zero shift the first and last window
+ * along that axis are partial. This is the same partition as rolling the
+ * grid by the shift and masking wrapped-around pairs. Each token attends to
+ * the tokens of its own window only, per head:
+ *     out_i = sum_j softmax_j(q_i . k_j / sqrt(headdim)) v_j
+ * with no mask inside a window and no position bias.
+ *
+ * Layouts: q, k, v, out : (batch, T, H, W, nheads, headdim), dtype,
+ *   16-byte aligned.
+ * Supported: headdim in {16, 32, 64, 128}, Tw*Sw*Sw <= 512.
+ * Returns MATE_OK, MATE_ERR_INVALID_ARG, MATE_ERR_UNSUPPORTED or
+ *   MATE_ERR_CUDA.
+ */
+int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, int Tw, int Sw,
+             const int shift[3], void *out, const mate_attn_dims *d, void *stream);
+
+/*
+ * Debug export of the scan order the kernels use: out_dev[n] = grid offset
+ * of the n-th token of the scan (flip != 0: of the flipped scan). out_dev
+ * holds T*H*W int32 (device memory, caller-owned).
+ */
+int mate_debug_rms_map(int T, int H, int W, int scan_mode, int flip, int32_t *out_dev, void *stream);
+
+/*
+ * Debug export of the TESA window partition the kernels use: out_win_dev[g]
+ * = window id of grid token g, windows numbered in (t, h, w) order of their
+ * first token. out_win_dev holds T*H*W int32 (device memory, caller-owned).
+ */
+int mate_debug_tesa_map(int T, int H, int W, int Tw, int Sw, const int shift[3], int32_t *out_win_dev,
+                        void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device-side error word
+ * that kernels set when a bounded wait gives up (MATE_ERR_TIMEOUT) or a
+ * device-side check fails (MATE_ERR_INVALID_ARG). Returns MATE_ERR_CUDA if
+ * the synchronisation itself fails.
+ */
+int mate_last_error(void *stream);
+
+/*
+ * Phases of a call, reported to the phase hook below. Each phase is one
+ * kernel launch.
+ */
+#define MATE_PHASE_REVIEW_POOL 1 /* average-pool x, dt, B over the review boxes   */
+#define MATE_PHASE_REVIEW_SCAN 2 /* scan the review prefix -> its final state      */
+#define MATE_PHASE_CHUNK_STATE 3 /* chunk-local scan states                        */
+#define MATE_PHASE_STATE_PASS 4  /* chain chunk states -> state entering each chunk */
+#define MATE_PHASE_CHUNK_OUT 5   /* outputs of every chunk, both directions         */
+#define MATE_PHASE_TESA 6        /* windowed attention                             */
+
+/*
+ * Optional enqueue-time hook, for timing phases with events on the caller's
+ * stream: while set, the library calls fn(phase, is_end, stream, user) on the
+ * calling host thread right before (is_end = 0) and right after (is_end = 1)
+ * it enqueues each phase on `stream`. NULL removes the hook. Process-wide;
+ * set or clear it only while no other thread is calling into the library.
+ */
+typedef void (*mate_phase_hook)(int phase, int is_end, void *stream, void *user);
+void mate_set_phase_hook(mate_phase_hook fn, void *user);
+
+/* Number of kernels the library has launched since the process started. */
+uint64_t mate_kernel_launches(void);
+
+/* Static text for a status code. */
+const char *mate_status_string(int code);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int mate_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MATE_H */

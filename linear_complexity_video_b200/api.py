@@ -1,0 +1,151 @@
+"""Thin PyTorch-facing binding of the C ABI in include/mate.h.
+
+Each function marshals torch CUDA tensors into the pointers and sizes of the
+C entry point of the same name and raises ``MateError`` on a non-zero status.
+PyTorch supplies device memory and the current stream; every step of the
+computation runs in libmate.so. The ``bissd`` / ``tesa`` helpers read the
+dims off the tensor shapes and allocate the output and workspace with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import MATE_BF16, MATE_DIR_BI, MATE_F32, check, mate_attn_dims, mate_ssd_dims
+
+_DT = {torch.float32: MATE_F32, torch.bfloat16: MATE_BF16}
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _int3(v: Optional[Sequence[int]]):
+    if v is None:
+        return None
+    return (ctypes.c_int * 3)(*[int(u) for u in v])
+
+
+def _require(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def ssd_dims(batch, nheads, headdim, dstate, ngroups, chunk, dtype, directions=MATE_DIR_BI) -> mate_ssd_dims:
+    return mate_ssd_dims(batch, nheads, headdim, dstate, ngroups, chunk,
+                         _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype), directions)
+
+
+def attn_dims(batch, nheads, headdim, dtype) -> mate_attn_dims:
+    return mate_attn_dims(batch, nheads, headdim, _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype))
+
+
+# ---------------------------------------------------------------------------
+# the C entry points, one to one
+# ---------------------------------------------------------------------------
+def mate_bissd_workspace_bytes(T: int, H: int, W: int, review_pool, dims: mate_ssd_dims) -> int:
+    return int(_lib.load().mate_bissd_workspace_bytes(T, H, W, _int3(review_pool), ctypes.byref(dims)))
+
+
+def mate_bissd_fwd(x, dt, A, B, C, D, T, H, W, scan_mode, review_pool, out, dims: mate_ssd_dims,
+                   workspace: torch.Tensor, stream=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = _lib.load().mate_bissd_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), T, H, W, scan_mode,
+                                    _int3(review_pool), _ptr(out), ctypes.byref(dims), _ptr(workspace),
+                                    ctypes.c_size_t(ws_bytes), _stream_handle(stream))
+    check("mate_bissd_fwd", rc)
+
+
+def tesa_fwd(q, k, v, T, H, W, Tw, Sw, shift, out, dims: mate_attn_dims, stream=None) -> None:
+    rc = _lib.load().tesa_fwd(_ptr(q), _ptr(k), _ptr(v), T, H, W, Tw, Sw, _int3(shift), _ptr(out),
+                              ctypes.byref(dims), _stream_handle(stream))
+    check("tesa_fwd", rc)
+
+
+def mate_debug_rms_map(T, H, W, scan_mode, flip, out, stream=None) -> None:
+    check("mate_debug_rms_map",
+          _lib.load().mate_debug_rms_map(T, H, W, scan_mode, int(flip), _ptr(out), _stream_handle(stream)))
+
+
+def mate_debug_tesa_map(T, H, W, Tw, Sw, shift, out, stream=None) -> None:
+    check("mate_debug_tesa_map",
+          _lib.load().mate_debug_tesa_map(T, H, W, Tw, Sw, _int3(shift), _ptr(out), _stream_handle(stream)))
+
+
+def mate_last_error(stream=None) -> int:
+    return int(_lib.load().mate_last_error(_stream_handle(stream)))
+
+
+def mate_version() -> int:
+    return int(_lib.load().mate_version())
+
+
+# ---------------------------------------------------------------------------
+# shape-reading helpers
+# ---------------------------------------------------------------------------
+def bissd_workspace(x: torch.Tensor, B: torch.Tensor, review_pool=None, chunk: int = 256,
+                    directions: int = MATE_DIR_BI) -> torch.Tensor:
+    b, T, H, W, nh, P = x.shape
+    G, Ns = B.shape[4:]
+    dims = ssd_dims(b, nh, P, Ns, G, chunk, x.dtype, directions)
+    n = mate_bissd_workspace_bytes(T, H, W, review_pool, dims)
+    if n == 0:
+        raise ValueError("unsupported bi-SSD dims")
+    return torch.empty(n, dtype=torch.uint8, device=x.device)
+
+
+def bissd(x, dt, A, B, C, D, scan_mode: int, review_pool=None, chunk: int = 256, directions: int = MATE_DIR_BI,
+          out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """MA-branch token mix. x: (batch, T, H, W, nh, P); dt: (batch, T, H, W, nh) fp32;
+    A, D: (nh,) fp32; B, C: (batch, T, H, W, G, Ns). Returns out shaped like x."""
+    for t, n in ((x, "x"), (B, "B"), (C, "C")):
+        _require(t, n, x.dtype)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
+        _require(t, n, torch.float32)
+    b, T, H, W, nh, P = x.shape
+    G, Ns = B.shape[4:]
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = bissd_workspace(x, B, review_pool, chunk, directions)
+    dims = ssd_dims(b, nh, P, Ns, G, chunk, x.dtype, directions)
+    mate_bissd_fwd(x, dt, A, B, C, D, T, H, W, scan_mode, review_pool, out, dims, workspace, stream)
+    return out
+
+
+def tesa(q, k, v, Tw: int, Sw: int, shift=(0, 0, 0), out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """TE-branch window attention. q, k, v: (batch, T, H, W, nh, d). Returns out shaped like q."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, q.dtype)
+    b, T, H, W, nh, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    tesa_fwd(q, k, v, T, H, W, Tw, Sw, shift, out, attn_dims(b, nh, d, q.dtype), stream)
+    return out
+
+
+def rms_map(T: int, H: int, W: int, scan_mode: int, flip: bool = False, device="cuda") -> torch.Tensor:
+    out = torch.empty(T * H * W, dtype=torch.int32, device=device)
+    mate_debug_rms_map(T, H, W, scan_mode, flip, out)
+    return out
+
+
+def tesa_map(T: int, H: int, W: int, Tw: int, Sw: int, shift, device="cuda") -> torch.Tensor:
+    out = torch.empty(T * H * W, dtype=torch.int32, device=device)
+    mate_debug_tesa_map(T, H, W, Tw, Sw, shift, out)
+    return out

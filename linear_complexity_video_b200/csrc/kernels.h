@@ -1,0 +1,82 @@
+// Launch-side view of the MATE kernels: argument blocks filled by the C ABI
+// layer (mate_abi.cu) and the launchers each kernel file provides.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mate {
+
+// Everything one bi-SSD call needs, resolved on the host.
+struct SsdArgs {
+    const void *x;
+    const float *dt;
+    const float *A;
+    const void *B;
+    const void *C;
+    const float *D;
+    void *out;
+    int batch, T, H, W, N;   // grid; N = T*H*W tokens per batch element
+    int nh, P, Ns, G;        // heads, head dim, state size, B/C groups
+    int Q, nchunks;          // chunk length and chunk count of the scan
+    int mode;                // MATE_SCAN_*
+    int dirs;                // MATE_DIR_* bit mask (1 forward, 2 flipped)
+    int review;              // 1 when a review prefix precedes the scan
+    int pt, ph, pw;          // review pooling box
+    int Tp, Hp, Wp, Np;      // pooled grid and its token count
+    int bf16;                // 1: x, B, C, out are bf16; 0: fp32
+    // workspace carve-outs (fp32)
+    float *states_f;         // (batch, nh, nchunks, P, Ns): chunk-local forward states,
+                             //   overwritten by the state entering each chunk
+    float *states_b;         // same for the flipped scan
+    float *alpha;            // (batch, nh, nchunks): exp(A * sum of dt over the chunk)
+    float *h_init;           // (batch, nh, P, Ns): state after the review prefix
+    float *pooled;           // (batch, Np, nh*P + nh + G*Ns): pooled x, dt, B
+};
+
+struct TesaArgs {
+    const void *q;
+    const void *k;
+    const void *v;
+    void *out;
+    int batch, T, H, W, N;
+    int nh, d;
+    int Tw, Sw;
+    int st, sh, sw;          // shifts
+    int offt, offh, offw;    // window offsets (S - s) % S
+    int nwt, nwh, nww;       // windows per axis
+    int bf16;
+};
+
+// Phase hook and launch counter (mate_set_phase_hook / mate_kernel_launches).
+void phase_mark(int phase, int is_end, cudaStream_t s);
+void count_launch();
+
+// Brackets one phase's launch: reports it to the hook and counts the launch.
+struct Phase {
+    int phase;
+    cudaStream_t s;
+    Phase(int p, cudaStream_t st) : phase(p), s(st) { phase_mark(phase, 0, s); }
+    ~Phase()
+    {
+        count_launch();
+        phase_mark(phase, 1, s);
+    }
+};
+
+// Workspace layout of a bi-SSD call; offsets in bytes from the base pointer.
+struct SsdWorkspace {
+    size_t states_f, states_b, alpha, h_init, pooled, total;
+};
+SsdWorkspace ssd_workspace_layout(const SsdArgs &a);
+
+// generic CUDA-core bi-SSD path (any supported dims, fp32 or bf16)
+cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s);
+// generic CUDA-core TESA path
+cudaError_t launch_tesa_generic(const TesaArgs &a, cudaStream_t s);
+// debug maps
+cudaError_t launch_rms_map(int T, int H, int W, int mode, int flip, int32_t *out, cudaStream_t s);
+cudaError_t launch_tesa_map(const TesaArgs &a, int32_t *out, cudaStream_t s);
+
+}  // namespace mate

@@ -1,0 +1,288 @@
+// C ABI of the MATE token-mix library: argument checks, workspace layout and
+// dispatch to the kernels. Declarations and contracts live in include/mate.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "../../include/mate.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mate {
+
+// Device-side error word: kernels with bounded waits or device checks set it;
+// mate_last_error() reads and clears it.
+__device__ int g_error_word = 0;
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+mate_phase_hook g_hook = nullptr;
+void *g_hook_user = nullptr;
+}  // namespace
+
+void phase_mark(int phase, int is_end, cudaStream_t s)
+{
+    if (g_hook) g_hook(phase, is_end, static_cast<void *>(s), g_hook_user);
+}
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr int kMaxChunk = 256;
+constexpr size_t kAlign = 256;
+constexpr size_t kMaxSmem = 227 * 1024;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool supported_head(int v) { return v == 16 || v == 32 || v == 64; }
+
+// Fill the shape part of SsdArgs and check it; returns MATE_OK or an error.
+int ssd_shape(int T, int H, int W, const int *pool, const mate_ssd_dims *d, int scan_mode, SsdArgs &a)
+{
+    if (!d) return MATE_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || W <= 0 || d->batch <= 0 || d->nheads <= 0 || d->ngroups <= 0 || d->chunk <= 0)
+        return MATE_ERR_INVALID_ARG;
+    const int64_t N = (int64_t)T * H * W;
+    if (N >= ((int64_t)1 << 31) || N * d->batch >= ((int64_t)1 << 40)) return MATE_ERR_INVALID_ARG;
+    if (d->nheads % d->ngroups) return MATE_ERR_INVALID_ARG;
+    if (scan_mode < 0 || scan_mode > 3) return MATE_ERR_INVALID_ARG;
+    const int dirs = d->directions == 0 ? MATE_DIR_BI : d->directions;
+    if (dirs < 1 || dirs > 3) return MATE_ERR_INVALID_ARG;
+    if (d->dtype != MATE_F32 && d->dtype != MATE_BF16) return MATE_ERR_UNSUPPORTED;
+    if (!supported_head(d->headdim) || !supported_head(d->dstate)) return MATE_ERR_UNSUPPORTED;
+    if (d->chunk > kMaxChunk) return MATE_ERR_UNSUPPORTED;
+    memset(&a, 0, sizeof(a));
+    a.batch = d->batch;
+    a.T = T;
+    a.H = H;
+    a.W = W;
+    a.N = (int)N;
+    a.nh = d->nheads;
+    a.P = d->headdim;
+    a.Ns = d->dstate;
+    a.G = d->ngroups;
+    a.Q = d->chunk;
+    a.nchunks = (int)((N + d->chunk - 1) / d->chunk);
+    a.mode = scan_mode;
+    a.dirs = dirs;
+    a.bf16 = d->dtype == MATE_BF16;
+    const bool review = pool && (pool[0] || pool[1] || pool[2]);
+    if (review) {
+        if (pool[0] <= 0 || pool[1] <= 0 || pool[2] <= 0) return MATE_ERR_INVALID_ARG;
+        if (T % pool[0] || H % pool[1] || W % pool[2]) return MATE_ERR_INVALID_ARG;
+        a.review = 1;
+        a.pt = pool[0];
+        a.ph = pool[1];
+        a.pw = pool[2];
+        a.Tp = T / pool[0];
+        a.Hp = H / pool[1];
+        a.Wp = W / pool[2];
+        a.Np = a.Tp * a.Hp * a.Wp;
+    }
+    return MATE_OK;
+}
+
+void carve(SsdArgs &a, void *ws)
+{
+    const SsdWorkspace l = ssd_workspace_layout(a);
+    char *base = static_cast<char *>(ws);
+    a.states_f = reinterpret_cast<float *>(base + l.states_f);
+    a.states_b = reinterpret_cast<float *>(base + l.states_b);
+    a.alpha = reinterpret_cast<float *>(base + l.alpha);
+    a.h_init = a.review ? reinterpret_cast<float *>(base + l.h_init) : nullptr;
+    a.pooled = a.review ? reinterpret_cast<float *>(base + l.pooled) : nullptr;
+}
+
+int attn_shape(int T, int H, int W, int Tw, int Sw, const int *shift, const mate_attn_dims *d, TesaArgs &a)
+{
+    if (!d || !shift) return MATE_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || W <= 0 || Tw <= 0 || Sw <= 0 || d->batch <= 0 || d->nheads <= 0)
+        return MATE_ERR_INVALID_ARG;
+    const int64_t N = (int64_t)T * H * W;
+    if (N >= ((int64_t)1 << 31)) return MATE_ERR_INVALID_ARG;
+    if (shift[0] < 0 || shift[0] >= Tw || shift[1] < 0 || shift[1] >= Sw || shift[2] < 0 || shift[2] >= Sw)
+        return MATE_ERR_INVALID_ARG;
+    if (d->dtype != MATE_F32 && d->dtype != MATE_BF16) return MATE_ERR_UNSUPPORTED;
+    memset(&a, 0, sizeof(a));
+    a.batch = d->batch;
+    a.T = T;
+    a.H = H;
+    a.W = W;
+    a.N = (int)N;
+    a.nh = d->nheads;
+    a.d = d->headdim;
+    a.Tw = Tw;
+    a.Sw = Sw;
+    a.st = shift[0];
+    a.sh = shift[1];
+    a.sw = shift[2];
+    a.offt = win_offset(Tw, shift[0]);
+    a.offh = win_offset(Sw, shift[1]);
+    a.offw = win_offset(Sw, shift[2]);
+    a.nwt = (T + a.offt + Tw - 1) / Tw;
+    a.nwh = (H + a.offh + Sw - 1) / Sw;
+    a.nww = (W + a.offw + Sw - 1) / Sw;
+    a.bf16 = d->dtype == MATE_BF16;
+    return MATE_OK;
+}
+
+}  // namespace
+
+SsdWorkspace ssd_workspace_layout(const SsdArgs &a)
+{
+    SsdWorkspace l;
+    const size_t nstate = (size_t)a.batch * a.nh * a.nchunks * a.P * a.Ns;
+    size_t off = 0;
+    l.states_f = off;
+    off = align_up(off + nstate * sizeof(float));
+    l.states_b = off;
+    off = align_up(off + nstate * sizeof(float));
+    l.alpha = off;
+    off = align_up(off + (size_t)a.batch * a.nh * a.nchunks * sizeof(float));
+    l.h_init = off;
+    if (a.review) off = align_up(off + (size_t)a.batch * a.nh * a.P * a.Ns * sizeof(float));
+    l.pooled = off;
+    if (a.review)
+        off = align_up(off + (size_t)a.batch * a.Np * ((size_t)a.nh * a.P + a.nh + (size_t)a.G * a.Ns) * sizeof(float));
+    l.total = off;
+    return l;
+}
+
+}  // namespace mate
+
+using namespace mate;
+
+extern "C" {
+
+size_t mate_bissd_workspace_bytes(int T, int H, int W, const int review_pool[3], const mate_ssd_dims *d)
+{
+    SsdArgs a;
+    if (ssd_shape(T, H, W, review_pool, d, MATE_SCAN_SR, a) != MATE_OK) return 0;
+    return ssd_workspace_layout(a).total;
+}
+
+int mate_bissd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D,
+                   int T, int H, int W, int scan_mode, const int review_pool[3], void *out, const mate_ssd_dims *d,
+                   void *workspace, size_t ws_bytes, void *stream)
+{
+    SsdArgs a;
+    int rc = ssd_shape(T, H, W, review_pool, d, scan_mode, a);
+    if (rc != MATE_OK) return rc;
+    if (!x || !dt || !A || !B || !C || !D || !out) return MATE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(out, 16) || !aligned(dt, 4) ||
+        !aligned(A, 4) || !aligned(D, 4))
+        return MATE_ERR_INVALID_ARG;
+    const size_t e = a.bf16 ? 2 : 4;
+    const size_t ntok = (size_t)a.batch * a.N;
+    const size_t xbytes = ntok * a.nh * a.P * e, bbytes = ntok * a.G * a.Ns * e;
+    if (overlaps(out, xbytes, x, xbytes) || overlaps(out, xbytes, B, bbytes) || overlaps(out, xbytes, C, bbytes) ||
+        overlaps(out, xbytes, dt, ntok * a.nh * 4) || overlaps(out, xbytes, A, a.nh * 4) ||
+        overlaps(out, xbytes, D, a.nh * 4))
+        return MATE_ERR_INVALID_ARG;
+    const SsdWorkspace l = ssd_workspace_layout(a);
+    if (!workspace || ws_bytes < l.total || !aligned(workspace, kAlign)) return MATE_ERR_WORKSPACE;
+    if (overlaps(workspace, l.total, out, xbytes) || overlaps(workspace, l.total, x, xbytes))
+        return MATE_ERR_INVALID_ARG;
+    a.x = x;
+    a.dt = dt;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.D = D;
+    a.out = out;
+    carve(a, workspace);
+    const size_t smem = ((size_t)a.Q * (a.P + a.Ns) + 2 * a.P * a.Ns + 3 * (size_t)a.Q) * sizeof(float);
+    if (smem > kMaxSmem) return MATE_ERR_UNSUPPORTED;
+    cudaError_t err = launch_ssd_generic(a, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
+int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, int Tw, int Sw, const int shift[3],
+             void *out, const mate_attn_dims *d, void *stream)
+{
+    TesaArgs a;
+    int rc = attn_shape(T, H, W, Tw, Sw, shift, d, a);
+    if (rc != MATE_OK) return rc;
+    if (a.d != 16 && a.d != 32 && a.d != 64 && a.d != 128) return MATE_ERR_UNSUPPORTED;
+    const size_t e = a.bf16 ? 2 : 4;
+    const size_t maxm = (size_t)Tw * Sw * Sw;
+    if (maxm > 512 || 2 * maxm * a.d * e + maxm * 4 > kMaxSmem) return MATE_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out) return MATE_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return MATE_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)a.batch * a.N * a.nh * a.d * e;
+    if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) || overlaps(out, bytes, v, bytes))
+        return MATE_ERR_INVALID_ARG;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.out = out;
+    cudaError_t err = launch_tesa_generic(a, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
+int mate_debug_rms_map(int T, int H, int W, int scan_mode, int flip, int32_t *out_dev, void *stream)
+{
+    if (T <= 0 || H <= 0 || W <= 0 || scan_mode < 0 || scan_mode > 3 || !out_dev) return MATE_ERR_INVALID_ARG;
+    if ((int64_t)T * H * W >= ((int64_t)1 << 31)) return MATE_ERR_INVALID_ARG;
+    cudaError_t err = launch_rms_map(T, H, W, scan_mode, flip, out_dev, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
+int mate_debug_tesa_map(int T, int H, int W, int Tw, int Sw, const int shift[3], int32_t *out_win_dev, void *stream)
+{
+    mate_attn_dims d = {1, 1, 16, MATE_F32};
+    TesaArgs a;
+    int rc = attn_shape(T, H, W, Tw, Sw, shift, &d, a);
+    if (rc != MATE_OK) return rc;
+    if (!out_win_dev) return MATE_ERR_INVALID_ARG;
+    cudaError_t err = launch_tesa_map(a, out_win_dev, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
+int mate_last_error(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MATE_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return MATE_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return MATE_ERR_CUDA;
+    }
+    return word;
+}
+
+const char *mate_status_string(int code)
+{
+    switch (code) {
+    case MATE_OK: return "ok";
+    case MATE_ERR_INVALID_ARG: return "invalid argument";
+    case MATE_ERR_UNSUPPORTED: return "unsupported dims or dtype";
+    case MATE_ERR_CUDA: return "CUDA error";
+    case MATE_ERR_TIMEOUT: return "bounded device wait timed out";
+    case MATE_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    default: return "unknown status";
+    }
+}
+
+int mate_version(void) { return 100; }
+
+void mate_set_phase_hook(mate_phase_hook fn, void *user)
+{
+    g_hook = fn;
+    g_hook_user = user;
+}
+
+uint64_t mate_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,387 @@
+// Bidirectional Mamba2 (SSD) scan in Rotary Major Scan order with review
+// tokens: CUDA-core path for any supported head size, fp32 or bf16 storage.
+//
+// Method (paper review "LinGen ...", section 三, MA-Branch items 1-3): per
+// head, s_n = exp(dt_n A) s_{n-1} + dt_n x_n B_n^T and y_n = s_n C_n + D x_n,
+// scanned over the RMS-ordered sequence and over its flip; the flipped
+// outputs are flipped back and added. Review tokens prepend a pooled copy of
+// the grid and its flip.
+//
+// Decomposition (the chunked "state-space duality" form of Mamba2). The
+// sequence is cut into chunks of Q tokens. Inside a chunk, with
+// cum_i = A * sum_{k<=i} dt_k and excl_i = cum_i - A dt_i (both from the
+// chunk start), the forward direction contributes
+//     sum_{j<=i} (C_i.B_j) exp(cum_i - cum_j) dt_j x_j + exp(cum_i) C_i S_in
+// and the flipped direction, written in original order,
+//     sum_{j>=i} (C_i.B_j) exp(excl_j - excl_i) dt_j x_j + exp(cum_end - excl_i) C_i S'_in
+// where S_in is the forward state entering the chunk from the left and S'_in
+// the flipped-scan state entering it from the right. The review prefix reads
+// the same in both directions, so both scans start from the one state it
+// leaves behind (h_init).
+//
+// Kernels:
+//   review_pool   average-pool x, dt, B over each pooling box
+//   review_scan   scan the prefix [R, flip(R)] from zero -> h_init
+//   chunk_state   chunk-local forward and flipped states and chunk decay
+//   state_pass    chain the chunk states: state entering every chunk
+//   chunk_out     intra-chunk quadratic term + entering states + D x
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mate {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTile = 32;
+
+__device__ __forceinline__ size_t tok_index(const SsdArgs &a, int b, int g) { return (size_t)b * a.N + g; }
+
+// ---------------------------------------------------------------------------
+// review_pool: pooled[b][cell][ch] = mean over the cell's box of x | dt | B
+// grid: (Np, ceil(channels / 256), batch)
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) review_pool_kernel(SsdArgs a)
+{
+    const int cell = blockIdx.x, b = blockIdx.z;
+    const int CX = a.nh * a.P, CD = a.nh, CB = a.G * a.Ns, CH = CX + CD + CB;
+    const int ch = blockIdx.y * blockDim.x + threadIdx.x;
+    if (ch >= CH) return;
+    const int hw = a.Hp * a.Wp;
+    const int tp = cell / hw, r = cell - tp * hw, hp = r / a.Wp, wp = r - hp * a.Wp;
+    const T *x = static_cast<const T *>(a.x);
+    const T *Bm = static_cast<const T *>(a.B);
+    float sum = 0.f;
+    for (int i = 0; i < a.pt; ++i)
+        for (int j = 0; j < a.ph; ++j)
+            for (int k = 0; k < a.pw; ++k) {
+                const int g = ((tp * a.pt + i) * a.H + hp * a.ph + j) * a.W + wp * a.pw + k;
+                const size_t tok = tok_index(a, b, g);
+                if (ch < CX)
+                    sum += ld(x + tok * CX + ch);
+                else if (ch < CX + CD)
+                    sum += a.dt[tok * CD + (ch - CX)];
+                else
+                    sum += ld(Bm + tok * CB + (ch - CX - CD));
+            }
+    a.pooled[((size_t)b * a.Np + cell) * CH + ch] = sum / (float)(a.pt * a.ph * a.pw);
+}
+
+// ---------------------------------------------------------------------------
+// review_scan: h_init[b][h] = state after scanning [R, flip(R)] from zero,
+// R = pooled grid in scan order. grid: (nh, batch)
+// ---------------------------------------------------------------------------
+template <int P, int NS>
+__global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
+{
+    constexpr int PN = P * NS;
+    constexpr int E = (PN + kThreads - 1) / kThreads;
+    __shared__ float xs[kTile][P];
+    __shared__ float bs[kTile][NS];
+    __shared__ float ds[kTile];
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int grp = h / (a.nh / a.G);
+    const int CX = a.nh * a.P, CD = a.nh, CH = CX + CD + a.G * a.Ns;
+    const float Ah = a.A[h];
+    const int L = 2 * a.Np;
+    float s[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[e] = 0.f;
+    for (int base = 0; base < L; base += kTile) {
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < kTile * (P + NS + 1); idx += blockDim.x) {
+            const int k = idx / (P + NS + 1), c = idx - k * (P + NS + 1);
+            const int pos = base + k;
+            if (pos >= L) continue;
+            const int r = pos < a.Np ? pos : L - 1 - pos;  // [R, flip(R)]
+            const int cell = rms_grid_offset(r, a.Tp, a.Hp, a.Wp, a.mode);
+            const float *row = a.pooled + ((size_t)b * a.Np + cell) * CH;
+            if (c < P)
+                xs[k][c] = row[h * P + c];
+            else if (c < P + NS)
+                bs[k][c - P] = row[CX + CD + grp * NS + (c - P)];
+            else
+                ds[k] = row[CX + h];
+        }
+        __syncthreads();
+        const int kmax = min(kTile, L - base);
+        for (int k = 0; k < kmax; ++k) {
+            const float dk = ds[k];
+            const float dec = expf(dk * Ah);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int idx = threadIdx.x + e * kThreads;
+                if (idx < PN) {
+                    const int p = idx / NS, n = idx - p * NS;
+                    s[e] = dec * s[e] + dk * xs[k][p] * bs[k][n];
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int idx = threadIdx.x + e * kThreads;
+        if (idx < PN) a.h_init[((size_t)b * a.nh + h) * PN + idx] = s[e];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// chunk_state: chunk-local states from a zero start
+//   forward : sum_j exp(cum_end - cum_j) dt_j x_j B_j^T
+//   flipped : sum_j exp(excl_j) dt_j x_j B_j^T
+//   alpha   : exp(cum_end)
+// grid: (nchunks, nh, batch)
+// ---------------------------------------------------------------------------
+template <typename T, int P, int NS>
+__global__ void __launch_bounds__(kThreads) chunk_state_kernel(SsdArgs a)
+{
+    constexpr int PN = P * NS;
+    constexpr int E = (PN + kThreads - 1) / kThreads;
+    __shared__ float cum[256];
+    __shared__ float dts[256];
+    __shared__ int goff[256];
+    __shared__ float xs[kTile][P];
+    __shared__ float bs[kTile][NS];
+    __shared__ float wf[kTile], wb[kTile];
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n0 = c * a.Q, len = min(a.Q, a.N - n0);
+    const int grp = h / (a.nh / a.G);
+    const float Ah = a.A[h];
+    const T *x = static_cast<const T *>(a.x);
+    const T *Bm = static_cast<const T *>(a.B);
+    for (int i = threadIdx.x; i < len; i += blockDim.x) {
+        const int g = rms_grid_offset(n0 + i, a.T, a.H, a.W, a.mode);
+        goff[i] = g;
+        const float d = a.dt[tok_index(a, b, g) * a.nh + h];
+        dts[i] = d;
+        cum[i] = d * Ah;
+    }
+    block_inclusive_scan(cum, len);
+    const float cend = cum[len - 1];
+    float sf[E], sb[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) sf[e] = sb[e] = 0.f;
+    for (int base = 0; base < len; base += kTile) {
+        const int kmax = min(kTile, len - base);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < kTile * (P + NS); idx += blockDim.x) {
+            const int k = idx / (P + NS), col = idx - k * (P + NS);
+            if (k >= kmax) continue;
+            const size_t tok = tok_index(a, b, goff[base + k]);
+            if (col < P)
+                xs[k][col] = ld(x + (tok * a.nh + h) * P + col);
+            else
+                bs[k][col - P] = ld(Bm + (tok * a.G + grp) * NS + (col - P));
+        }
+        if (threadIdx.x < kmax) {
+            const int i = base + threadIdx.x;
+            wf[threadIdx.x] = expf(cend - cum[i]) * dts[i];
+            wb[threadIdx.x] = expf(cum[i] - dts[i] * Ah) * dts[i];
+        }
+        __syncthreads();
+        for (int k = 0; k < kmax; ++k) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int idx = threadIdx.x + e * kThreads;
+                if (idx < PN) {
+                    const int p = idx / NS, n = idx - p * NS;
+                    const float v = xs[k][p] * bs[k][n];
+                    sf[e] += wf[k] * v;
+                    sb[e] += wb[k] * v;
+                }
+            }
+        }
+    }
+    const size_t base_out = (((size_t)b * a.nh + h) * a.nchunks + c) * PN;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int idx = threadIdx.x + e * kThreads;
+        if (idx < PN) {
+            a.states_f[base_out + idx] = sf[e];
+            a.states_b[base_out + idx] = sb[e];
+        }
+    }
+    if (threadIdx.x == 0) a.alpha[((size_t)b * a.nh + h) * a.nchunks + c] = expf(cend);
+}
+
+// ---------------------------------------------------------------------------
+// state_pass: replace every chunk-local state by the state entering that
+// chunk (forward: from the left; flipped: from the right). Both start from
+// h_init with review tokens, else from zero. grid: (nh, batch, 2)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) state_pass_kernel(SsdArgs a)
+{
+    const int h = blockIdx.x, b = blockIdx.y, dir = blockIdx.z;
+    if (!(a.dirs & (1 << dir))) return;
+    const int PN = a.P * a.Ns, nc = a.nchunks;
+    float *S = (dir == 0 ? a.states_f : a.states_b) + ((size_t)b * a.nh + h) * nc * PN;
+    const float *al = a.alpha + ((size_t)b * a.nh + h) * nc;
+    for (int idx = threadIdx.x; idx < PN; idx += blockDim.x) {
+        float Hv = a.review ? a.h_init[((size_t)b * a.nh + h) * PN + idx] : 0.f;
+        if (dir == 0) {
+            float nxt = S[idx];
+            for (int c = 0; c < nc; ++c) {
+                const float cur = nxt;
+                if (c + 1 < nc) nxt = S[(size_t)(c + 1) * PN + idx];
+                S[(size_t)c * PN + idx] = Hv;
+                Hv = al[c] * Hv + cur;
+            }
+        } else {
+            float nxt = S[(size_t)(nc - 1) * PN + idx];
+            for (int c = nc - 1; c >= 0; --c) {
+                const float cur = nxt;
+                if (c > 0) nxt = S[(size_t)(c - 1) * PN + idx];
+                S[(size_t)c * PN + idx] = Hv;
+                Hv = al[c] * Hv + cur;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// chunk_out: one thread per token of the chunk.
+// grid: (nchunks, nh, batch); block: 256; dynamic shared memory:
+//   bs[Q][NS] xs[Q][P] Hf[P][NS] Hb[P][NS] cum[Q] dts[Q] goff[Q]
+// ---------------------------------------------------------------------------
+template <typename T, int P, int NS>
+__global__ void __launch_bounds__(kThreads) chunk_out_kernel(SsdArgs a)
+{
+    extern __shared__ float smem[];
+    const int Q = a.Q;
+    float *bs = smem;
+    float *xs = bs + (size_t)Q * NS;
+    float *Hf = xs + (size_t)Q * P;
+    float *Hb = Hf + P * NS;
+    float *cum = Hb + P * NS;
+    float *dts = cum + Q;
+    int *goff = reinterpret_cast<int *>(dts + Q);
+
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n0 = c * Q, len = min(Q, a.N - n0);
+    const int grp = h / (a.nh / a.G);
+    const float Ah = a.A[h], Dh = a.D[h];
+    const bool fwd = a.dirs & 1, bwd = a.dirs & 2;
+    const T *x = static_cast<const T *>(a.x);
+    const T *Bm = static_cast<const T *>(a.B);
+    const T *Cm = static_cast<const T *>(a.C);
+    T *out = static_cast<T *>(a.out);
+
+    for (int i = threadIdx.x; i < len; i += blockDim.x) {
+        const int g = rms_grid_offset(n0 + i, a.T, a.H, a.W, a.mode);
+        goff[i] = g;
+        const float d = a.dt[tok_index(a, b, g) * a.nh + h];
+        dts[i] = d;
+        cum[i] = d * Ah;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < len * (P + NS); idx += blockDim.x) {
+        const int i = idx / (P + NS), col = idx - i * (P + NS);
+        const size_t tok = tok_index(a, b, goff[i]);
+        if (col < P)
+            xs[i * P + col] = ld(x + (tok * a.nh + h) * P + col);
+        else
+            bs[i * NS + (col - P)] = ld(Bm + (tok * a.G + grp) * NS + (col - P));
+    }
+    const size_t sbase = (((size_t)b * a.nh + h) * a.nchunks + c) * (P * NS);
+    for (int idx = threadIdx.x; idx < P * NS; idx += blockDim.x) {
+        Hf[idx] = fwd ? a.states_f[sbase + idx] : 0.f;
+        Hb[idx] = bwd ? a.states_b[sbase + idx] : 0.f;
+    }
+    block_inclusive_scan(cum, len);
+
+    const int i = threadIdx.x;
+    if (i >= len) return;
+    const size_t tok = tok_index(a, b, goff[i]);
+    float ci[NS];
+#pragma unroll
+    for (int n = 0; n < NS; ++n) ci[n] = ld(Cm + (tok * a.G + grp) * NS + n);
+    float y[P];
+#pragma unroll
+    for (int p = 0; p < P; ++p) y[p] = 0.f;
+    const float cum_i = cum[i];
+    const float excl_i = cum_i - dts[i] * Ah;
+    const float cend = cum[len - 1];
+    for (int j = 0; j < len; ++j) {
+        float w = 0.f;
+        if (fwd && j <= i) w += expf(cum_i - cum[j]);
+        if (bwd && j >= i) w += expf((cum[j] - dts[j] * Ah) - excl_i);
+        if (w == 0.f) continue;
+        float s = 0.f;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) s += ci[n] * bs[j * NS + n];
+        w *= s * dts[j];
+#pragma unroll
+        for (int p = 0; p < P; ++p) y[p] += w * xs[j * P + p];
+    }
+    const float rf = fwd ? expf(cum_i) : 0.f;
+    const float rb = bwd ? expf(cend - excl_i) : 0.f;
+    const float dx = (float)((int)fwd + (int)bwd) * Dh;
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        float zf = 0.f, zb = 0.f;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+            zf += ci[n] * Hf[p * NS + n];
+            zb += ci[n] * Hb[p * NS + n];
+        }
+        y[p] += rf * zf + rb * zb + dx * xs[i * P + p];
+    }
+    T *o = out + (tok * a.nh + h) * P;
+#pragma unroll
+    for (int p = 0; p < P; ++p) st(o + p, y[p]);
+}
+
+template <typename T, int P, int NS>
+cudaError_t run(const SsdArgs &a, cudaStream_t s)
+{
+    const size_t smem = ((size_t)a.Q * (P + NS) + 2 * P * NS + 3 * (size_t)a.Q) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(chunk_out_kernel<T, P, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    if (a.review) {
+        const int CH = a.nh * a.P + a.nh + a.G * a.Ns;
+        {
+            Phase ph(MATE_PHASE_REVIEW_POOL, s);
+            review_pool_kernel<T><<<dim3(a.Np, (CH + kThreads - 1) / kThreads, a.batch), kThreads, 0, s>>>(a);
+        }
+        {
+            Phase ph(MATE_PHASE_REVIEW_SCAN, s);
+            review_scan_kernel<P, NS><<<dim3(a.nh, a.batch), kThreads, 0, s>>>(a);
+        }
+    }
+    {
+        Phase ph(MATE_PHASE_CHUNK_STATE, s);
+        chunk_state_kernel<T, P, NS><<<dim3(a.nchunks, a.nh, a.batch), kThreads, 0, s>>>(a);
+    }
+    {
+        Phase ph(MATE_PHASE_STATE_PASS, s);
+        state_pass_kernel<<<dim3(a.nh, a.batch, 2), kThreads, 0, s>>>(a);
+    }
+    {
+        Phase ph(MATE_PHASE_CHUNK_OUT, s);
+        chunk_out_kernel<T, P, NS><<<dim3(a.nchunks, a.nh, a.batch), kThreads, smem, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch_dims(const SsdArgs &a, cudaStream_t s)
+{
+#define MATE_CASE(PP, NN) \
+    if (a.P == PP && a.Ns == NN) return run<T, PP, NN>(a, s);
+    MATE_CASE(16, 16) MATE_CASE(16, 32) MATE_CASE(16, 64)
+    MATE_CASE(32, 16) MATE_CASE(32, 32) MATE_CASE(32, 64)
+    MATE_CASE(64, 16) MATE_CASE(64, 32) MATE_CASE(64, 64)
+#undef MATE_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s)
+{
+    return a.bf16 ? dispatch_dims<__nv_bfloat16>(a, s) : dispatch_dims<float>(a, s);
+}
+
+}  // namespace mate

@@ -1,0 +1,111 @@
+"""The C ABI library: it loads, exports every declared symbol and rejects bad
+arguments on the host (no GPU needed: these calls return before touching
+CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_complexity_video_b200 as mate
+from linear_complexity_video_b200 import _lib, api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = "\n".join(ln for ln in src.splitlines() if not ln.lstrip().startswith(("typedef", "#")))
+            names.update(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(\w+)\s*\(", src, flags=re.M))
+    return names
+
+
+def test_library_loads():
+    L = mate.load()
+    assert mate.mate_version() >= 100
+    assert L.mate_status_string(0) == b"ok"
+
+
+def test_every_declared_symbol_is_exported():
+    L = mate.load()
+    names = declared_functions()
+    assert {"mate_bissd_fwd", "tesa_fwd", "mate_bissd_workspace_bytes"} <= names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert set(_lib.EXPORTS) == names, "binding list and header disagree"
+
+
+def _dims(**kw):
+    base = dict(batch=1, nheads=2, headdim=16, dstate=16, ngroups=1, chunk=32, dtype=0, directions=3)
+    base.update(kw)
+    return _lib.mate_ssd_dims(**base)
+
+
+def test_workspace_query_rejects_bad_dims():
+    ok = api.mate_bissd_workspace_bytes(4, 8, 8, (2, 4, 4), _dims())
+    assert ok > 0
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, (3, 4, 4), _dims()) == 0      # pool does not divide T
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(headdim=48)) == 0  # unsupported head dim
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(nheads=3, ngroups=2)) == 0
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(chunk=512)) == 0
+    assert api.mate_bissd_workspace_bytes(0, 8, 8, None, _dims()) == 0
+
+
+def test_workspace_grows_linearly_in_tokens():
+    d = _dims(nheads=80, headdim=64, dstate=64, chunk=256, dtype=1)
+    w1 = api.mate_bissd_workspace_bytes(32, 32, 32, None, d)
+    w4 = api.mate_bissd_workspace_bytes(128, 32, 32, None, d)
+    assert abs(w4 / w1 - 4.0) < 0.01
+
+
+def _call_bissd(L, ptr=1, T=4, dims=None, ws=1 << 20, ws_ptr=256, mode=0, pool=None, align=256):
+    p = ctypes.c_void_p(ptr * align)
+    f = ctypes.c_void_p(ptr * align + (1 << 30))
+    dims = dims or _dims()
+    pool_arr = (ctypes.c_int * 3)(*pool) if pool else None
+    out = ctypes.c_void_p((ptr * align + (2 << 30)) if ptr else 0)
+    return L.mate_bissd_fwd(p, f, f, p, p, f, T, 8, 8, mode, pool_arr, out, ctypes.byref(dims),
+                            ctypes.c_void_p(ws_ptr + (3 << 30) if ws_ptr else 0), ctypes.c_size_t(ws), None)
+
+
+def test_bissd_argument_errors_on_host():
+    L = mate.load()
+    assert _call_bissd(L, ptr=0) == _lib.MATE_ERR_INVALID_ARG                      # null pointers
+    assert _call_bissd(L, mode=7) == _lib.MATE_ERR_INVALID_ARG                     # bad scan mode
+    assert _call_bissd(L, pool=(3, 4, 4)) == _lib.MATE_ERR_INVALID_ARG             # pool must divide
+    assert _call_bissd(L, dims=_dims(dtype=5)) == _lib.MATE_ERR_UNSUPPORTED
+    assert _call_bissd(L, align=2) == _lib.MATE_ERR_INVALID_ARG                    # misaligned x
+    assert _call_bissd(L, ws=16) == _lib.MATE_ERR_WORKSPACE                        # workspace too small
+    assert _call_bissd(L, ws_ptr=0) == _lib.MATE_ERR_WORKSPACE                     # no workspace
+
+
+def test_tesa_argument_errors_on_host():
+    L = mate.load()
+    d = _lib.mate_attn_dims(1, 2, 16, 0)
+    p = ctypes.c_void_p(1 << 20)
+    o = ctypes.c_void_p(1 << 32)
+    sh = lambda *v: (ctypes.c_int * 3)(*v)
+    assert L.tesa_fwd(p, p, p, 4, 8, 8, 2, 4, sh(2, 0, 0), o, ctypes.byref(d), None) == _lib.MATE_ERR_INVALID_ARG
+    assert L.tesa_fwd(p, p, p, 4, 8, 8, 2, 4, sh(0, -1, 0), o, ctypes.byref(d), None) == _lib.MATE_ERR_INVALID_ARG
+    assert L.tesa_fwd(p, p, p, 4, 8, 8, 2, 4, None, o, ctypes.byref(d), None) == _lib.MATE_ERR_INVALID_ARG
+    d48 = _lib.mate_attn_dims(1, 2, 48, 0)
+    assert L.tesa_fwd(p, p, p, 4, 8, 8, 2, 4, sh(0, 0, 0), o, ctypes.byref(d48), None) == _lib.MATE_ERR_UNSUPPORTED
+    # out overlapping q
+    assert L.tesa_fwd(p, p, p, 4, 8, 8, 2, 4, sh(0, 0, 0), p, ctypes.byref(d), None) == _lib.MATE_ERR_INVALID_ARG
+
+
+def test_debug_map_argument_errors_on_host():
+    L = mate.load()
+    assert L.mate_debug_rms_map(4, 8, 8, 9, 0, ctypes.c_void_p(256), None) == _lib.MATE_ERR_INVALID_ARG
+    assert L.mate_debug_rms_map(4, 8, 8, 0, 0, None, None) == _lib.MATE_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(ImportError):
+        _lib.load()
