@@ -107,11 +107,14 @@ def test_bissd_directions_add_up():
     f = mate.bissd(*args, chunk=32, directions=1)
     b = mate.bissd(*args, chunk=32, directions=2)
     assert rel_err(host64(f + b), host64(bi)) <= 1e-6
-    # the flipped scan of a grid equals the forward scan of the grid reversed on every axis
+    # Without review tokens, the flipped scan of a grid equals the forward scan of the grid
+    # reversed on every axis. (With review tokens it does not: reversing the grid reverses R,
+    # and the prefix [flip(R), R] differs from [R, flip(R)].)
     rev = lambda t: t.flip(1, 2, 3).contiguous()
-    fr = mate.bissd(rev(dev["x"]), rev(dev["dt"]), dev["A"], rev(dev["B"]), rev(dev["C"]), dev["D"], 3, cfg.review,
+    b0 = mate.bissd(*args[:7], None, chunk=32, directions=2)
+    fr = mate.bissd(rev(dev["x"]), rev(dev["dt"]), dev["A"], rev(dev["B"]), rev(dev["C"]), dev["D"], 3, None,
                     chunk=32, directions=1)
-    assert rel_err(host64(rev(fr)), host64(b)) <= 1e-5
+    assert rel_err(host64(rev(fr)), host64(b0)) <= 1e-5
 
 
 def test_bissd_256p_bf16():
