@@ -138,6 +138,38 @@ int mate_bissd_fwd(const void *x, const float *dt, const float *A, const void *B
                    void *out, const mate_ssd_dims *d, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Allocation-free variant of mate_bissd_fwd. The paper has no counterpart:
+ * this is a deployment aid of this library.
+ *
+ * Who needs it: callers that cannot allocate device memory on their call
+ * path, such as a plugin inside a host application that owns the whole
+ * device memory pool, code that must not pay the implicit device
+ * synchronisation of cudaMalloc/cudaFree, or a process whose device memory
+ * budget is fixed up front. They pass inputs and outputs only; the scratch
+ * that mate_bissd_fwd takes as `workspace` comes from a fixed array of
+ * MATE_NOALLOC_SCRATCH_BYTES bytes that is part of the library's device
+ * image. Every GPU that loads the library holds that array until the
+ * process exits.
+ *
+ * Arguments, layouts and results are those of mate_bissd_fwd.
+ * - Returns MATE_ERR_WORKSPACE, enqueueing nothing, when
+ *   mate_bissd_workspace_bytes(...) for these dims exceeds
+ *   MATE_NOALLOC_SCRATCH_BYTES.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ * - All calls share the one array, which keeps the last call's contents.
+ *   Calls whose work may overlap on the GPU (e.g. on unordered streams) race
+ *   on it and must be serialised by the caller. Nothing needs clearing
+ *   between calls: the kernels write every scratch word before reading it.
+ * - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define MATE_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+int mate_bissd_fwd_noalloc(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                           const float *D, int T, int H, int W, int scan_mode, const int review_pool[3],
+                           void *out, const mate_ssd_dims *d, void *stream);
+
+/*
  * TE-branch: TEmporal Swin Attention (paper review, TE-Branch; the superapi
  * product page, "Technical Principles": windows shift between layers).
  *

@@ -35,7 +35,10 @@ EXPORTS = (
     "mate_version",
     "mate_set_phase_hook",
     "mate_kernel_launches",
+    "mate_bissd_fwd_noalloc",
 )
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 PHASES = {1: "review_pool", 2: "review_scan", 3: "chunk_state", 4: "state_pass", 5: "chunk_out", 6: "tesa"}
 PHASE_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
@@ -90,6 +93,9 @@ def load() -> ctypes.CDLL:
     L.mate_version.restype = ctypes.c_int
     L.mate_set_phase_hook.argtypes = [PHASE_HOOK, ctypes.c_void_p]
     L.mate_set_phase_hook.restype = None
+    L.mate_bissd_fwd_noalloc.argtypes = [_vp] * 6 + [ctypes.c_int] * 4 + [_ip, _vp, ctypes.POINTER(mate_ssd_dims),
+                                                                            _vp]
+    L.mate_bissd_fwd_noalloc.restype = ctypes.c_int
     L.mate_kernel_launches.argtypes = []
     L.mate_kernel_launches.restype = ctypes.c_uint64
     _lib = L

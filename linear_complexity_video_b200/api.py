@@ -71,6 +71,15 @@ def mate_bissd_fwd(x, dt, A, B, C, D, T, H, W, scan_mode, review_pool, out, dims
     check("mate_bissd_fwd", rc)
 
 
+def mate_bissd_fwd_noalloc(x, dt, A, B, C, D, T, H, W, scan_mode, review_pool, out, dims: mate_ssd_dims,
+                           stream=None) -> None:
+    """mate_bissd_fwd with the library's fixed scratch array instead of a caller workspace."""
+    rc = _lib.load().mate_bissd_fwd_noalloc(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), T, H, W,
+                                            scan_mode, _int3(review_pool), _ptr(out), ctypes.byref(dims),
+                                            _stream_handle(stream))
+    check("mate_bissd_fwd_noalloc", rc)
+
+
 def tesa_fwd(q, k, v, T, H, W, Tw, Sw, shift, out, dims: mate_attn_dims, stream=None) -> None:
     rc = _lib.load().tesa_fwd(_ptr(q), _ptr(k), _ptr(v), T, H, W, Tw, Sw, _int3(shift), _ptr(out),
                               ctypes.byref(dims), _stream_handle(stream))
