@@ -33,6 +33,7 @@ struct SsdArgs {
     float *alpha;            // (batch, nh, nchunks): exp(A * sum of dt over the chunk)
     float *h_init;           // (batch, nh, P, Ns): state after the review prefix
     float *pooled;           // (batch, Np, nh*P + nh + G*Ns): pooled x, dt, B
+    int *err;                // device error word (MATE_ERR_* set by bounded waits)
 };
 
 struct TesaArgs {
@@ -47,6 +48,7 @@ struct TesaArgs {
     int offt, offh, offw;    // window offsets (S - s) % S
     int nwt, nwh, nww;       // windows per axis
     int bf16;
+    int *err;                // device error word
 };
 
 // Phase hook and launch counter (mate_set_phase_hook / mate_kernel_launches).
@@ -73,8 +75,16 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a);
 
 // generic CUDA-core bi-SSD path (any supported dims, fp32 or bf16)
 cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s);
+// the generic review, chunk-state and state-chain kernels for bf16, head dim 64, d_state 64
+cudaError_t launch_ssd_prepass_bf16_64(const SsdArgs &a, cudaStream_t s);
 // generic CUDA-core TESA path
 cudaError_t launch_tesa_generic(const TesaArgs &a, cudaStream_t s);
+// tensor-core TESA path (bf16, head dim 128, 128-token windows)
+bool tesa_tc_supported(const TesaArgs &a);
+cudaError_t launch_tesa_tc(const TesaArgs &a, cudaStream_t s);
+// tensor-core bi-SSD path (bf16, head dim 64, d_state 64, both directions)
+bool ssd_tc_supported(const SsdArgs &a);
+cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s);
 // debug maps
 cudaError_t launch_rms_map(int T, int H, int W, int mode, int flip, int32_t *out, cudaStream_t s);
 cudaError_t launch_tesa_map(const TesaArgs &a, int32_t *out, cudaStream_t s);

@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "../../include/mate.h"
 #include "common.cuh"
@@ -22,6 +23,22 @@ mate_phase_hook g_hook = nullptr;
 void *g_hook_user = nullptr;
 }  // namespace
 
+// Device address of g_error_word on the current device (looked up once per device).
+int *error_word_ptr()
+{
+    static std::mutex mu;
+    static int *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
+}
+
 void phase_mark(int phase, int is_end, cudaStream_t s)
 {
     if (g_hook) g_hook(phase, is_end, static_cast<void *>(s), g_hook_user);
@@ -31,7 +48,8 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 
-constexpr int kMaxChunk = 256;
+constexpr int kMaxChunk = 1024;        // longest chunk the state kernels take
+constexpr int kMaxGenericChunk = 256;  // longest chunk of the CUDA-core output kernel
 constexpr size_t kAlign = 256;
 constexpr size_t kMaxSmem = 227 * 1024;
 
@@ -91,6 +109,16 @@ int ssd_shape(int T, int H, int W, const int *pool, const mate_ssd_dims *d, int 
         a.Np = a.Tp * a.Hp * a.Wp;
     }
     return MATE_OK;
+}
+
+// 1 when the tensor-core path runs these dims, 0 when the CUDA-core path does,
+// -1 when neither can.
+int ssd_path(const SsdArgs &a)
+{
+    if (ssd_tc_supported(a)) return 1;
+    const size_t smem = ((size_t)a.Q * (a.P + a.Ns) + 2 * a.P * a.Ns + 3 * (size_t)a.Q) * sizeof(float);
+    if (a.Q > kMaxGenericChunk || smem > kMaxSmem) return -1;
+    return 0;
 }
 
 void carve(SsdArgs &a, void *ws)
@@ -169,6 +197,7 @@ size_t mate_bissd_workspace_bytes(int T, int H, int W, const int review_pool[3],
 {
     SsdArgs a;
     if (ssd_shape(T, H, W, review_pool, d, MATE_SCAN_SR, a) != MATE_OK) return 0;
+    if (ssd_path(a) < 0) return 0;
     return ssd_workspace_layout(a).total;
 }
 
@@ -179,6 +208,8 @@ int mate_bissd_fwd(const void *x, const float *dt, const float *A, const void *B
     SsdArgs a;
     int rc = ssd_shape(T, H, W, review_pool, d, scan_mode, a);
     if (rc != MATE_OK) return rc;
+    const int path = ssd_path(a);
+    if (path < 0) return MATE_ERR_UNSUPPORTED;
     if (!x || !dt || !A || !B || !C || !D || !out) return MATE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(out, 16) || !aligned(dt, 4) ||
         !aligned(A, 4) || !aligned(D, 4))
@@ -202,9 +233,10 @@ int mate_bissd_fwd(const void *x, const float *dt, const float *A, const void *B
     a.D = D;
     a.out = out;
     carve(a, workspace);
-    const size_t smem = ((size_t)a.Q * (a.P + a.Ns) + 2 * a.P * a.Ns + 3 * (size_t)a.Q) * sizeof(float);
-    if (smem > kMaxSmem) return MATE_ERR_UNSUPPORTED;
-    cudaError_t err = launch_ssd_generic(a, static_cast<cudaStream_t>(stream));
+    a.err = error_word_ptr();
+    if (!a.err) return MATE_ERR_CUDA;
+    const cudaError_t err = path == 1 ? launch_ssd_tc(a, static_cast<cudaStream_t>(stream))
+                                      : launch_ssd_generic(a, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
 }
 
@@ -227,7 +259,10 @@ int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, i
     a.k = k;
     a.v = v;
     a.out = out;
-    cudaError_t err = launch_tesa_generic(a, static_cast<cudaStream_t>(stream));
+    a.err = error_word_ptr();
+    if (!a.err) return MATE_ERR_CUDA;
+    cudaError_t err = tesa_tc_supported(a) ? launch_tesa_tc(a, static_cast<cudaStream_t>(stream))
+                                           : launch_tesa_generic(a, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
 }
 

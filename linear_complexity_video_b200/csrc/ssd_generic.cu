@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTile = 32;
+constexpr int kMaxStateChunk = 1024;  // chunk_state handles chunks of up to this many tokens
 
 __device__ __forceinline__ size_t tok_index(const SsdArgs &a, int b, int g) { return (size_t)b * a.N + g; }
 
@@ -138,9 +139,9 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(SsdArgs a)
 {
     constexpr int PN = P * NS;
     constexpr int E = (PN + kThreads - 1) / kThreads;
-    __shared__ float cum[256];
-    __shared__ float dts[256];
-    __shared__ int goff[256];
+    __shared__ float cum[kMaxStateChunk];
+    __shared__ float dts[kMaxStateChunk];
+    __shared__ int goff[kMaxStateChunk];
     __shared__ float xs[kTile][P];
     __shared__ float bs[kTile][NS];
     __shared__ float wf[kTile], wb[kTile];
@@ -332,13 +333,11 @@ __global__ void __launch_bounds__(kThreads) chunk_out_kernel(SsdArgs a)
     for (int p = 0; p < P; ++p) st(o + p, y[p]);
 }
 
+// review prefix, chunk-local states and the state chain: everything before
+// the chunk outputs
 template <typename T, int P, int NS>
-cudaError_t run(const SsdArgs &a, cudaStream_t s)
+cudaError_t run_prepass(const SsdArgs &a, cudaStream_t s)
 {
-    const size_t smem = ((size_t)a.Q * (P + NS) + 2 * P * NS + 3 * (size_t)a.Q) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(chunk_out_kernel<T, P, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
     if (a.review) {
         const int CH = a.nh * a.P + a.nh + a.G * a.Ns;
         {
@@ -358,6 +357,18 @@ cudaError_t run(const SsdArgs &a, cudaStream_t s)
         Phase ph(MATE_PHASE_STATE_PASS, s);
         state_pass_kernel<<<dim3(a.nh, a.batch, 2), kThreads, 0, s>>>(a);
     }
+    return cudaGetLastError();
+}
+
+template <typename T, int P, int NS>
+cudaError_t run(const SsdArgs &a, cudaStream_t s)
+{
+    const size_t smem = ((size_t)a.Q * (P + NS) + 2 * P * NS + 3 * (size_t)a.Q) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(chunk_out_kernel<T, P, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    e = run_prepass<T, P, NS>(a, s);
+    if (e != cudaSuccess) return e;
     {
         Phase ph(MATE_PHASE_CHUNK_OUT, s);
         chunk_out_kernel<T, P, NS><<<dim3(a.nchunks, a.nh, a.batch), kThreads, smem, s>>>(a);
@@ -382,6 +393,11 @@ cudaError_t dispatch_dims(const SsdArgs &a, cudaStream_t s)
 cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s)
 {
     return a.bf16 ? dispatch_dims<__nv_bfloat16>(a, s) : dispatch_dims<float>(a, s);
+}
+
+cudaError_t launch_ssd_prepass_bf16_64(const SsdArgs &a, cudaStream_t s)
+{
+    return run_prepass<__nv_bfloat16, 64, 64>(a, s);
 }
 
 }  // namespace mate

@@ -51,7 +51,12 @@ def test_workspace_query_rejects_bad_dims():
     assert api.mate_bissd_workspace_bytes(4, 8, 8, (3, 4, 4), _dims()) == 0      # pool does not divide T
     assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(headdim=48)) == 0  # unsupported head dim
     assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(nheads=3, ngroups=2)) == 0
-    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(chunk=512)) == 0
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(chunk=512)) == 0   # CUDA-core path: chunk <= 256
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(chunk=2048)) == 0
+    # the bf16, 64 x 64 tensor-core path takes chunks of 128..512 tokens
+    tc = dict(nheads=4, headdim=64, dstate=64, dtype=1)
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(chunk=512, **tc)) > 0
+    assert api.mate_bissd_workspace_bytes(4, 8, 8, None, _dims(chunk=640, **tc)) == 0
     assert api.mate_bissd_workspace_bytes(0, 8, 8, None, _dims()) == 0
 
 
