@@ -75,8 +75,8 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a);
 
 // generic CUDA-core bi-SSD path (any supported dims, fp32 or bf16)
 cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s);
-// the generic review, chunk-state and state-chain kernels for bf16, head dim 64, d_state 64
-cudaError_t launch_ssd_prepass_bf16_64(const SsdArgs &a, cudaStream_t s);
+// the generic review pooling and prefix scan for bf16, head dim 64, d_state 64
+cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s);
 // generic CUDA-core TESA path
 cudaError_t launch_tesa_generic(const TesaArgs &a, cudaStream_t s);
 // tensor-core TESA path (bf16, head dim 128, 128-token windows)

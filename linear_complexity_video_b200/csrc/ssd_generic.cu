@@ -70,6 +70,73 @@ __global__ void __launch_bounds__(kThreads) review_pool_kernel(SsdArgs a)
 }
 
 // ---------------------------------------------------------------------------
+// review_pool, vectorised for bf16 storage: each thread sums one 16-byte vector
+// (8 channels of x or B) or one float4 of dt over the cell's box, with four
+// independent partial sums per channel for memory-level parallelism.
+// grid: (Np, ceil(vectors / 256), batch); needs nh*P % 8 == 0, G*Ns % 8 == 0,
+// nh % 4 == 0 and a 16-byte aligned dt.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
+{
+    const int cell = blockIdx.x, b = blockIdx.z;
+    const int CX = a.nh * a.P, CD = a.nh, CB = a.G * a.Ns, CH = CX + CD + CB;
+    const int VX = CX / 8, VB = CB / 8, VD = CD / 4;
+    const int v = blockIdx.y * blockDim.x + threadIdx.x;
+    if (v >= VX + VB + VD) return;
+    const int hw = a.Hp * a.Wp;
+    const int tp = cell / hw, r = cell - tp * hw, hp = r / a.Wp, wp = r - hp * a.Wp;
+    const int box = a.pt * a.ph * a.pw;
+    const int kind = v < VX ? 0 : (v < VX + VB ? 1 : 2);
+    float acc[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+    for (int i0 = 0; i0 < box; i0 += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            if (i >= box) break;
+            const int it = i / (a.ph * a.pw), rr = i - it * (a.ph * a.pw), ih = rr / a.pw, iw = rr - ih * a.pw;
+            const int g = ((tp * a.pt + it) * a.H + hp * a.ph + ih) * a.W + wp * a.pw + iw;
+            const size_t tok = (size_t)b * a.N + g;
+            if (kind == 2) {
+                const float4 d = *reinterpret_cast<const float4 *>(a.dt + tok * CD + (v - VX - VB) * 4);
+                acc[u][0] += d.x;
+                acc[u][1] += d.y;
+                acc[u][2] += d.z;
+                acc[u][3] += d.w;
+            } else {
+                const __nv_bfloat16 *src = kind == 0 ? static_cast<const __nv_bfloat16 *>(a.x) + tok * CX + v * 8
+                                                     : static_cast<const __nv_bfloat16 *>(a.B) + tok * CB + (v - VX) * 8;
+                const uint4 q = *reinterpret_cast<const uint4 *>(src);
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[e]));
+                    acc[u][2 * e] += f.x;
+                    acc[u][2 * e + 1] += f.y;
+                }
+            }
+        }
+    }
+    const float inv = 1.f / (float)box;
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * inv;
+    float *dst = a.pooled + ((size_t)b * a.Np + cell) * CH;
+    if (kind == 0) {
+        dst += v * 8;
+    } else if (kind == 1) {
+        dst += CX + CD + (v - VX) * 8;
+    } else {
+        dst += CX + (v - VX - VB) * 4;
+    }
+    const int n = kind == 2 ? 4 : 8;
+    for (int e = 0; e < n; ++e) dst[e] = out[e];
+}
+
+// ---------------------------------------------------------------------------
 // review_scan: h_init[b][h] = state after scanning [R, flip(R)] from zero,
 // R = pooled grid in scan order. grid: (nh, batch)
 // ---------------------------------------------------------------------------
@@ -395,9 +462,25 @@ cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s)
     return a.bf16 ? dispatch_dims<__nv_bfloat16>(a, s) : dispatch_dims<float>(a, s);
 }
 
-cudaError_t launch_ssd_prepass_bf16_64(const SsdArgs &a, cudaStream_t s)
+cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)
 {
-    return run_prepass<__nv_bfloat16, 64, 64>(a, s);
+    const int CH = a.nh * a.P + a.nh + a.G * a.Ns;
+    const bool vec = (a.nh * a.P) % 8 == 0 && (a.G * a.Ns) % 8 == 0 && a.nh % 4 == 0 &&
+                     reinterpret_cast<uintptr_t>(a.dt) % 16 == 0;  // dt is read as float4
+    {
+        Phase ph(MATE_PHASE_REVIEW_POOL, s);
+        if (vec) {
+            const int nv = a.nh * a.P / 8 + a.G * a.Ns / 8 + a.nh / 4;
+            review_pool_vec_kernel<<<dim3(a.Np, (nv + kThreads - 1) / kThreads, a.batch), kThreads, 0, s>>>(a);
+        } else {
+            review_pool_kernel<__nv_bfloat16><<<dim3(a.Np, (CH + kThreads - 1) / kThreads, a.batch), kThreads, 0, s>>>(a);
+        }
+    }
+    {
+        Phase ph(MATE_PHASE_REVIEW_SCAN, s);
+        review_scan_kernel<64, 64><<<dim3(a.nh, a.batch), kThreads, 0, s>>>(a);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace mate

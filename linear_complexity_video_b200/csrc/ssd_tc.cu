@@ -1,36 +1,41 @@
-// Chunk outputs of the bidirectional SSD scan on the 5th-generation tensor
-// cores (tcgen05 + TMEM) for bf16 storage, head dim 64, d_state 64.
+// Bidirectional SSD scan on the 5th-generation tensor cores (tcgen05 + TMEM)
+// for bf16 storage, head dim 64, d_state 64.
 //
 // Method (paper review "LinGen ...", section 三, MA-Branch items 1-2): per
 // head, the Mamba2 recurrence s_n = exp(dt_n A) s_{n-1} + dt_n x_n B_n^T,
 // y_n = s_n C_n + D x_n, over the Rotary-Major-Scan sequence and over its
-// flip, flipped back and added.
+// flip, flipped back and added. The RMS order enters only through gather
+// addresses: row j of a chunk is the grid token of scan position start + j.
 //
-// One CTA per (head, chunk of L = 128*K tokens, batch element); the states
-// entering the chunk from the left (forward scan) and from the right (flipped
-// scan) come from the chunk-state chain. Inside the chunk, K sub-chunks of
-// 128 tokens:
-//   phase 1  for each sub-chunk, both sub-chunk-local states in one MMA:
-//            [ (w_f x)^T ; (w_b x)^T ] (128 x 128 tokens) . B (128 tokens x 64)
-//            with w_f[j] = exp(c_end - c_j) dt_j and w_b[j] = exp(e_j) dt_j
-//            (c: inclusive, e: exclusive cumulative sum of A dt inside the
-//            sub-chunk), rows 0-63 forward, rows 64-127 flipped, kept in TMEM.
-//   phase 2  chain them in TMEM: each lane owns one state row; the forward
-//            lanes walk the sub-chunks left to right, the flipped lanes right
-//            to left, replacing every local state by the state entering it.
-//   phase 3  for each sub-chunk, S = C B^T (128 x 128) into TMEM; thread i
-//            turns row i of S into row i of
-//               A = [ M | R_f C | R_b C ]   (128 x 256, bf16)
-//            with M_ij = S_ij dt_j (exp(c_i - c_j) [j <= i] + exp(e_j - e_i) [j >= i]),
-//            R_f[i] = exp(c_i), R_b[i] = exp(c_end - e_i); then one accumulating
-//            MMA chain computes A . [ x ; h_f^T ; h_b^T ] (256 x 64), and the
-//            epilogue adds 2 D x and stores the row to its grid position.
-// The exponentials of M are factored around the sub-chunk midpoint,
-// exp(c_i - c_j) = exp(c_i - r) exp(r - c_j), so a row costs two exps per
-// element pair only when the sub-chunk's decay range is too wide for fp32
-// (then every element is exponentiated exactly).
-// The RMS order enters only through the gather addresses: row j of a
-// sub-chunk is the grid token of scan position n = chunk start + j.
+// Three kernels, all with one CTA per (head, chunk of L = 128*K tokens, batch
+// element) where a chunk is processed as K sub-chunks of 128 tokens:
+//
+// chunk_state  chunk-local states of both directions from a zero start,
+//              one accumulating MMA per sub-chunk
+//                  [ (w_f x)^T ; (w_b x)^T ] (128 x 128 tokens) . B (128 tokens x 64)
+//              with w_f[j] = exp(c_end - c_j) dt_j and w_b[j] = exp(e_j) dt_j
+//              (c, e: inclusive / exclusive cumulative sums of A dt over the
+//              chunk); rows 0-63 forward, rows 64-127 flipped.
+// state_chain  one thread per state element replaces every chunk-local state
+//              by the state entering the chunk (forward from the left, flipped
+//              from the right), starting from the review state or zero.
+// chunk_out    phase 1: the same MMA per sub-chunk with sub-chunk-local
+//              weights, each result kept in its own TMEM slot;
+//              phase 2: chain the slots in TMEM from the chunk's entering
+//              states (each lane owns a state row; forward lanes walk left to
+//              right, flipped lanes right to left);
+//              phase 3: per sub-chunk, S = C B^T (128 x 128) into TMEM; row i
+//              of S becomes row i of A = [ M | R_f C | R_b C ] (128 x 256) with
+//                  M_ij = S_ij dt_j (exp(c_i - c_j) [j <= i] + exp(e_j - e_i) [j >= i]),
+//                  R_f[i] = exp(c_i), R_b[i] = exp(c_end - e_i),
+//              and one accumulating MMA chain computes A . [ x ; h_f^T ; h_b^T ];
+//              the epilogue adds 2 D x and stores each row at its grid position.
+// The exponentials of M are factored around the sub-chunk midpoint r,
+// exp(c_i - c_j) = exp(c_i - r) exp(r - c_j), whenever the sub-chunk's decay
+// range fits fp32; otherwise every element is exponentiated exactly.
+//
+// 256 threads per CTA: thread t works on row r = t % 128 (TMEM lane r) and
+// half g = t / 128 of that row's columns.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -39,74 +44,36 @@ namespace mate {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kSub = 128;        // tokens per sub-chunk
 constexpr int kMaxSubs = 4;      // sub-chunks per chunk held in TMEM
+constexpr int kMaxChunk = kSub * kMaxSubs;
 constexpr uint32_t kTile = 16384;
 
-// shared memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffX = 0;                 // 2 buffers x 16 KB
-constexpr uint32_t kOffB = 2 * kTile;         // 2 buffers
-constexpr uint32_t kOffC = 4 * kTile;         // 2 buffers
-constexpr uint32_t kOffA = 6 * kTile;         // 4 tiles: phase 1 U_f, U_b; phase 3 M0, M1, Cf, Cb
-constexpr uint32_t kOffH = 10 * kTile;        // h_f (8 KB) then h_b (8 KB)
-constexpr uint32_t kOffF = 11 * kTile;        // fp32 / int arrays
-constexpr int kMaxChunk = kSub * kMaxSubs;
-// arrays after kOffF: dt[512], cum[512] (inclusive, sub-chunk local), goff[512],
-// gf[128], gb[128], misc
-constexpr uint32_t kOffDt = kOffF;
-constexpr uint32_t kOffCum = kOffDt + kMaxChunk * 4;
-constexpr uint32_t kOffGoff = kOffCum + kMaxChunk * 4;
-constexpr uint32_t kOffGf = kOffGoff + kMaxChunk * 4;
-constexpr uint32_t kOffGb = kOffGf + kSub * 4;
-constexpr uint32_t kOffRed = kOffGb + kSub * 4;     // 8 floats of block reductions
-constexpr uint32_t kOffBar = kOffRed + 64;
-constexpr uint32_t kSmemUsed = kOffBar + 64;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
+constexpr float kFactorLimit = 80.f;  // |exponent| bound for the factored exps
 
-// TMEM columns
-constexpr uint32_t kColS = kMaxSubs * 64;   // S (128 cols) after the K state slots
-constexpr uint32_t kColAcc = kColS + 128;   // output accumulator (64 cols)
-constexpr uint32_t kTmemCols = 512;
+// ---------------------------------------------------------------------------
+// helpers shared by the kernels
+// ---------------------------------------------------------------------------
 
-constexpr float kFactorLimit = 80.f;        // |exponent| bound for the factored exps
-
-struct Smem {
-    uint8_t *base;
-    __device__ uint8_t *X(int buf) const { return base + kOffX + buf * kTile; }
-    __device__ uint8_t *B(int buf) const { return base + kOffB + buf * kTile; }
-    __device__ uint8_t *C(int buf) const { return base + kOffC + buf * kTile; }
-    __device__ uint8_t *A(int t) const { return base + kOffA + t * kTile; }
-    __device__ uint8_t *Hf() const { return base + kOffH; }
-    __device__ uint8_t *Hb() const { return base + kOffH + 8192; }
-    __device__ float *dt() const { return reinterpret_cast<float *>(base + kOffDt); }
-    __device__ float *cum() const { return reinterpret_cast<float *>(base + kOffCum); }
-    __device__ int *goff() const { return reinterpret_cast<int *>(base + kOffGoff); }
-    __device__ float *gf() const { return reinterpret_cast<float *>(base + kOffGf); }
-    __device__ float *gb() const { return reinterpret_cast<float *>(base + kOffGb); }
-    __device__ float *red() const { return reinterpret_cast<float *>(base + kOffRed); }
-    __device__ uint64_t *bar() const { return reinterpret_cast<uint64_t *>(base + kOffBar); }
-    __device__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + kOffBar + 8); }
-    __device__ int *abort_flag() const { return reinterpret_cast<int *>(base + kOffBar + 12); }
-};
-
-// Gather the 128 token rows of sub-chunk `sub` into swizzled tiles (x: 64 head
-// dims of head h; B and C: 64 state dims of the head's group). Rows past the
+// Gather the 128 token rows of sub-chunk `sub` into swizzled tiles (x: the 64
+// head dims of head h; B and C: the 64 state dims of the head's group; tC may
+// be null). goff[n] is the grid offset of chunk position n; rows past the
 // sequence end are zero.
-__device__ __forceinline__ void load_rows(const SsdArgs &a, const Smem &sm, int b, int h, int grp, int n0, int len,
-                                          int sub, int buf, bool withC)
+__device__ __forceinline__ void load_rows(const SsdArgs &a, uint8_t *tX, uint8_t *tB, uint8_t *tC, const int *goff,
+                                          int b, int h, int grp, int len, int sub)
 {
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
     const __nv_bfloat16 *Bm = static_cast<const __nv_bfloat16 *>(a.B);
     const __nv_bfloat16 *Cm = static_cast<const __nv_bfloat16 *>(a.C);
-    const int ntiles = withC ? 3 : 2;
+    const int ntiles = tC ? 3 : 2;
     for (int idx = threadIdx.x; idx < ntiles * kSub * 8; idx += kThreads) {
         const int tile = idx / (kSub * 8);
-        const int r = (idx / 8) % kSub, c = idx % 8;
-        const int n = sub * kSub + r;  // position inside the chunk
-        uint8_t *dst = (tile == 0 ? sm.X(buf) : tile == 1 ? sm.B(buf) : sm.C(buf)) + tc::sw128(r, c);
+        const int r = (idx >> 3) & (kSub - 1), c = idx & 7;
+        const int n = sub * kSub + r;
+        uint8_t *dst = (tile == 0 ? tX : tile == 1 ? tB : tC) + tc::sw128(r, c);
         if (n < len) {
-            const size_t tok = (size_t)b * a.N + sm.goff()[n];
+            const size_t tok = (size_t)b * a.N + goff[n];
             const __nv_bfloat16 *src = tile == 0 ? x + (tok * a.nh + h) * 64 + c * 8
                                                  : (tile == 1 ? Bm : Cm) + (tok * a.G + grp) * 64 + c * 8;
             tc::cp_async16(dst, src);
@@ -136,7 +103,7 @@ __device__ __forceinline__ void row_chunk(const uint8_t *tile, int r, int c, flo
     f = tc::unpack_bf16(u.w); v[6] = f.x; v[7] = f.y;
 }
 
-__device__ __forceinline__ void put_chunk(uint8_t *tile, int r, int c, const float (&v)[8])
+__device__ __forceinline__ void put_chunk(uint8_t *tile, int r, int c, const float *v)
 {
     uint4 u;
     u.x = tc::pack_bf16(v[0], v[1]);
@@ -146,187 +113,252 @@ __device__ __forceinline__ void put_chunk(uint8_t *tile, int r, int c, const flo
     *reinterpret_cast<uint4 *>(tile + tc::sw128(r, c)) = u;
 }
 
-__device__ __forceinline__ float block_max128(float v, float *red)
+// max over the CTA (256 threads); `red` holds 8 floats
+__device__ __forceinline__ float block_max(float v, float *red)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     __syncthreads();
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
     __syncthreads();
-    return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    float m = red[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+    return m;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a, int nsub)
+// Per-chunk setup shared by chunk_state and chunk_out: grid offsets and dt of
+// the chunk's L positions (zero past the sequence end).
+__device__ __forceinline__ void load_chunk_meta(const SsdArgs &a, int b, int h, int n0, int len, int L, int *goff,
+                                                float *dt)
 {
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = tc::smem_u32(smem_raw);
-    Smem sm{smem_raw + ((1024u - (raw & 1023u)) & 1023u)};
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
-    const int L = nsub * kSub;
-    const int n0 = c * L, len = min(L, a.N - n0);
-    const int grp = h / (a.nh / a.G);
-    const float Ah = a.A[h], Dh = a.D[h];
-    uint64_t *bar = sm.bar();
-    int *abort_flag = sm.abort_flag();
-    uint32_t mma_phase = 0;
-
-    if (warp == 0) tc::tmem_alloc(sm.tmem_slot(), kTmemCols);
-    if (tid == 0) {
-        tc::mbar_init(bar, 1);
-        tc::fence_mbar_init();
-        *abort_flag = 0;
-    }
-    // scan positions -> grid offsets, dt, sub-chunk-local inclusive cumsum of A dt
-    for (int n = tid; n < L; n += kThreads) {
+    for (int n = threadIdx.x; n < L; n += kThreads) {
         float d = 0.f;
         int g = 0;
         if (n < len) {
             g = rms_grid_offset(n0 + n, a.T, a.H, a.W, a.mode);
             d = a.dt[((size_t)b * a.N + g) * a.nh + h];
         }
-        sm.goff()[n] = g;
-        sm.dt()[n] = d;
+        goff[n] = g;
+        dt[n] = d;
     }
+}
+
+// Inclusive cumulative sums of A*dt within each 128-token sub-chunk (warp w
+// scans sub-chunk w); with `chunk_level`, continued across sub-chunks.
+__device__ __forceinline__ void sub_cumsums(const float *dt, float *cum, float Ah, int nsub, bool chunk_level,
+                                            float *carry_out)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < nsub) {
+        float carry = 0.f;
+        for (int q = 0; q < kSub; q += 32) {
+            const int n = warp * kSub + q + lane;
+            const float v = warp_inclusive_scan(dt[n] * Ah) + carry;
+            cum[n] = v;
+            carry = __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) carry_out[warp] = carry;
+    }
+    __syncthreads();
+    if (chunk_level) {
+        for (int n = threadIdx.x; n < nsub * kSub; n += kThreads) {
+            float off = 0.f;
+            for (int w = 0; w < n / kSub; ++w) off += carry_out[w];
+            cum[n] += off;
+        }
+        __syncthreads();
+    }
+}
+
+// U_f row r = w_f[r] x_r and U_b row r = w_b[r] x_r for chunks [4g, 4g + 4)
+__device__ __forceinline__ void build_u(const uint8_t *tX, uint8_t *uf, uint8_t *ub, int r, int g, float wf, float wb)
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int ch = 4 * g + q;
+        float v[8], f[8], e[8];
+        row_chunk(tX, r, ch, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            f[u] = wf * v[u];
+            e[u] = wb * v[u];
+        }
+        put_chunk(uf, r, ch, f);
+        put_chunk(ub, r, ch, e);
+    }
+}
+
+// [U_f^T ; U_b^T] (MN-major, two 64-row groups) . B (MN-major), K = 128 tokens
+__device__ __forceinline__ void mma_states(uint32_t d_tmem, uint32_t uf_addr, uint32_t b_addr, bool accumulate)
+{
+    const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+        tc::mma_bf16(d_tmem, tc::sdesc_sw128(uf_addr + s * 2048, kTile, 1024),
+                     tc::sdesc_sw128(b_addr + s * 2048, kTile, 1024), idesc, accumulate || s > 0);
+}
+
+// Bounded wait for the next MMA completion on `bar`; on timeout every thread
+// returns false (after a second bounded wait for the MMAs in flight).
+__device__ __forceinline__ bool mma_wait(uint64_t *bar, uint32_t &phase, int *err, int *abort_flag)
+{
+    const bool ok = tc::mbar_wait(bar, phase & 1u, err);
+    ++phase;
+    if (!ok) atomicExch(abort_flag, 1);
+    __syncthreads();
+    if (*abort_flag) {
+        tc::mbar_wait(bar, (phase - 1) & 1u, nullptr);
+        return false;
+    }
+    tc::tc_fence_after();
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// chunk_out
+// ---------------------------------------------------------------------------
+constexpr uint32_t kOffX = 0;                 // 2 buffers x 16 KB
+constexpr uint32_t kOffB = 2 * kTile;         // 2 buffers
+constexpr uint32_t kOffC = 4 * kTile;         // 2 buffers
+constexpr uint32_t kOffA = 6 * kTile;         // 4 tiles: phase 1 U_f, U_b; phase 3 M0, M1, R_f C, R_b C
+constexpr uint32_t kOffH = 10 * kTile;        // h_f (8 KB) then h_b (8 KB)
+constexpr uint32_t kOffDt = 11 * kTile;
+constexpr uint32_t kOffCum = kOffDt + kMaxChunk * 4;
+constexpr uint32_t kOffGoff = kOffCum + kMaxChunk * 4;
+constexpr uint32_t kOffGf = kOffGoff + kMaxChunk * 4;
+constexpr uint32_t kOffGb = kOffGf + kSub * 4;
+constexpr uint32_t kOffRed = kOffGb + kSub * 4;  // 8 floats
+constexpr uint32_t kOffBar = kOffRed + 64;
+constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;
+
+constexpr uint32_t kColS = kMaxSubs * 64;  // S (128 cols) after the state slots
+constexpr uint32_t kColAcc = kColS + 128;  // output accumulator (64 cols)
+constexpr uint32_t kTmemCols = 512;
+
+__global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a, int nsub)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    auto sX = [base](int i) { return base + kOffX + i * kTile; };
+    auto sB = [base](int i) { return base + kOffB + i * kTile; };
+    auto sC = [base](int i) { return base + kOffC + i * kTile; };
+    uint8_t *sA = base + kOffA;
+    uint8_t *sHf = base + kOffH, *sHb = base + kOffH + 8192;
+    float *sdt = reinterpret_cast<float *>(base + kOffDt);
+    float *scum = reinterpret_cast<float *>(base + kOffCum);
+    int *sgoff = reinterpret_cast<int *>(base + kOffGoff);
+    float *sgf = reinterpret_cast<float *>(base + kOffGf);
+    float *sgb = reinterpret_cast<float *>(base + kOffGb);
+    float *sred = reinterpret_cast<float *>(base + kOffRed);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + kOffBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffBar + 8);
+    int *abort_flag = reinterpret_cast<int *>(base + kOffBar + 12);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int r = tid & (kSub - 1), g = tid >> 7;   // row / TMEM lane, column half
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
+    const int L = nsub * kSub;
+    const int n0 = c * L, len = min(L, a.N - n0);
+    const int grp = h / (a.nh / a.G);
+    const float Ah = a.A[h], Dh2 = 2.f * a.D[h];
+    uint32_t mma_phase = 0;
+
+    if (warp == 0) tc::tmem_alloc(tmem_slot, kTmemCols);
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::fence_mbar_init();
+        *abort_flag = 0;
+    }
+    load_chunk_meta(a, b, h, n0, len, L, sgoff, sdt);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    const uint32_t tmem = *sm.tmem_slot();
+    const uint32_t tmem = *tmem_slot;
+    sub_cumsums(sdt, scum, Ah, nsub, false, sred);
 
-    // sub-chunk-local inclusive cumsums: warp w scans sub-chunk w (nsub <= 4)
-    if (warp < nsub) {
-        float carry = 0.f;
-        for (int base = 0; base < kSub; base += 32) {
-            const int n = warp * kSub + base + (tid & 31);
-            float v = warp_inclusive_scan(sm.dt()[n] * Ah) + carry;
-            sm.cum()[n] = v;
-            carry = __shfl_sync(0xffffffffu, v, 31);
-        }
-    }
-    __syncthreads();
-
-    auto mma_wait = [&]() -> bool {
-        const bool ok = tc::mbar_wait(bar, mma_phase & 1u, a.err);
-        ++mma_phase;
-        if (!ok) atomicExch(abort_flag, 1);
-        __syncthreads();
-        if (*abort_flag) {
-            tc::mbar_wait(bar, (mma_phase - 1) & 1u, nullptr);
-            return false;
-        }
-        tc::tc_fence_after();
-        return true;
-    };
-
-    // ---------------- phase 1: sub-chunk-local states -> TMEM -------------------
-    load_rows(a, sm, b, h, grp, n0, len, 0, 0, false);
+    // ---------------- phase 1: sub-chunk-local states -> TMEM slots ---------------
+    load_rows(a, sX(0), sB(0), nullptr, sgoff, b, h, grp, len, 0);
     for (int k = 0; k < nsub; ++k) {
         const int buf = k & 1;
-        if (k + 1 < nsub) load_rows(a, sm, b, h, grp, n0, len, k + 1, buf ^ 1, false);
+        if (k + 1 < nsub) load_rows(a, sX(buf ^ 1), sB(buf ^ 1), nullptr, sgoff, b, h, grp, len, k + 1);
         wait_loads(k + 1 < nsub);
         __syncthreads();
         {
-            const int j = tid, n = k * kSub + j;
-            const float cj = sm.cum()[n], dj = sm.dt()[n];
-            const float cend = sm.cum()[k * kSub + kSub - 1];
-            const float wf = __expf(cend - cj) * dj;
-            const float wb = __expf(cj - dj * Ah) * dj;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                float v[8], uf[8], ub[8];
-                row_chunk(sm.X(buf), j, ch, v);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    uf[e] = wf * v[e];
-                    ub[e] = wb * v[e];
-                }
-                put_chunk(sm.A(0), j, ch, uf);
-                put_chunk(sm.A(1), j, ch, ub);
-            }
+            const int n = k * kSub + r;
+            const float cj = scum[n], dj = sdt[n], cend = scum[k * kSub + kSub - 1];
+            build_u(sX(buf), sA, sA + kTile, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc::tc_fence_after();
-            const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
-            const uint32_t a0 = tc::smem_u32(sm.A(0)), b0 = tc::smem_u32(sm.B(buf));
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                tc::mma_bf16(tmem + k * 64, tc::sdesc_sw128(a0 + s * 2048, kTile, 1024),
-                             tc::sdesc_sw128(b0 + s * 2048, kTile, 1024), idesc, s > 0);
+            mma_states(tmem + k * 64, tc::smem_u32(sA), tc::smem_u32(sB(buf)), false);
             tc::mma_commit(bar);
         }
-        if (!mma_wait()) goto cleanup;
+        if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
     }
 
-    // ---------------- phase 2: chain the sub-chunk states in TMEM ----------------
+    // ---------------- phase 2: chain the sub-chunk states in TMEM ------------------
     {
-        const bool fwd = warp < 2;
-        const int p = fwd ? tid : tid - 64;
-        const float *Hin = (fwd ? a.states_f : a.states_b) + ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + p) * 64;
-        float hv[2][32];
+        const bool fwd = r < 64;
+        const int p = fwd ? r : r - 64;
+        const float *Hin =
+            (fwd ? a.states_f : a.states_b) + ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + p) * 64 + 32 * g;
+        float hv[32];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            hv[0][q] = Hin[q];
-            hv[1][q] = Hin[32 + q];
+        for (int q = 0; q < 8; ++q) {
+            const float4 v = *reinterpret_cast<const float4 *>(Hin + 4 * q);
+            hv[4 * q] = v.x;
+            hv[4 * q + 1] = v.y;
+            hv[4 * q + 2] = v.z;
+            hv[4 * q + 3] = v.w;
         }
-        const uint32_t lane_base = (uint32_t)(warp * 32);
         for (int it = 0; it < nsub; ++it) {
             const int k = fwd ? it : nsub - 1 - it;
-            const float alpha = __expf(sm.cum()[k * kSub + kSub - 1]);
-            float t0[32], t1[32];
-            tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, k * 64), t0);
-            tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, k * 64 + 32), t1);
+            const float alpha = __expf(scum[k * kSub + kSub - 1]);
+            const uint32_t ta = tc::tmem_addr(tmem, lane_base, k * 64 + 32 * g);
+            float t0[32];
+            tc::tmem_ld32(ta, t0);
             tc::tmem_wait_ld();
-            tc::tmem_st32(tc::tmem_addr(tmem, lane_base, k * 64), hv[0]);
-            tc::tmem_st32(tc::tmem_addr(tmem, lane_base, k * 64 + 32), hv[1]);
+            tc::tmem_st32(ta, hv);
             tc::tmem_wait_st();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                hv[0][q] = fmaf(alpha, hv[0][q], t0[q]);
-                hv[1][q] = fmaf(alpha, hv[1][q], t1[q]);
-            }
+            for (int q = 0; q < 32; ++q) hv[q] = fmaf(alpha, hv[q], t0[q]);
         }
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
 
-    // ---------------- phase 3: outputs ------------------------------------------
-    load_rows(a, sm, b, h, grp, n0, len, 0, 0, true);
+    // ---------------- phase 3: outputs ---------------------------------------------
+    load_rows(a, sX(0), sB(0), sC(0), sgoff, b, h, grp, len, 0);
     for (int k = 0; k < nsub; ++k) {
         const int buf = k & 1;
-        if (k + 1 < nsub) load_rows(a, sm, b, h, grp, n0, len, k + 1, buf ^ 1, true);
-        // the state entering sub-chunk k: lanes 0-63 forward rows, 64-127 flipped rows -> bf16 operands
+        if (k + 1 < nsub) load_rows(a, sX(buf ^ 1), sB(buf ^ 1), sC(buf ^ 1), sgoff, b, h, grp, len, k + 1);
+        // entering states of sub-chunk k -> bf16 operands (row r: forward if r < 64)
         {
-            const uint32_t lane_base = (uint32_t)(warp * 32);
-            float t0[32], t1[32];
-            tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, k * 64), t0);
-            tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, k * 64 + 32), t1);
+            float t0[32];
+            tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, k * 64 + 32 * g), t0);
             tc::tmem_wait_ld();
-            uint8_t *ht = warp < 2 ? sm.Hf() : sm.Hb();
-            const int p = warp < 2 ? tid : tid - 64;
+            uint8_t *ht = r < 64 ? sHf : sHb;
+            const int p = r & 63;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                float v[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = t0[ch * 8 + e];
-                put_chunk(ht, p, ch, v);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = t1[ch * 8 + e];
-                put_chunk(ht, p, ch + 4, v);
-            }
+            for (int q = 0; q < 4; ++q) put_chunk(ht, p, 4 * g + q, t0 + 8 * q);
         }
-        // factors of the decay matrix for this sub-chunk, around r = cum at its midpoint
-        const int i = tid, n = k * kSub + i;
-        const float ci = sm.cum()[n], di = sm.dt()[n];
+        const int n = k * kSub + r;
+        const float ci = scum[n], di = sdt[n];
         const float ei = ci - di * Ah;
-        const float cend = sm.cum()[k * kSub + kSub - 1];
-        const float r = sm.cum()[k * kSub + kSub / 2 - 1];
-        sm.gf()[i] = __expf(r - ci) * di;   // forward column factor
-        sm.gb()[i] = __expf(ei - r) * di;   // flipped column factor
-        const float range = block_max128(fmaxf(fabsf(ci - r), fabsf(ei - r)), sm.red());
+        const float cend = scum[k * kSub + kSub - 1];
+        const float rmid = scum[k * kSub + kSub / 2 - 1];
+        if (g == 0) {
+            sgf[r] = __expf(rmid - ci) * di;  // forward column factor
+            sgb[r] = __expf(ei - rmid) * di;  // flipped column factor
+        }
+        const float range = block_max(g == 0 ? fmaxf(fabsf(ci - rmid), fabsf(ei - rmid)) : 0.f, sred);
         const bool factored = range <= kFactorLimit;
         wait_loads(k + 1 < nsub);
         tc::fence_proxy_async_smem();
@@ -337,56 +369,71 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
         if (tid == 0) {
             tc::tc_fence_after();
             const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 0);
-            const uint32_t c0 = tc::smem_u32(sm.C(buf)), b0 = tc::smem_u32(sm.B(buf));
+            const uint32_t c0 = tc::smem_u32(sC(buf)), b0 = tc::smem_u32(sB(buf));
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                tc::mma_bf16(tmem + kColS, tc::sdesc_sw128(c0 + s * 32, 16, 1024),
-                             tc::sdesc_sw128(b0 + s * 32, 16, 1024), idesc, s > 0);
+                tc::mma_bf16(tmem + kColS, tc::sdesc_sw128(c0 + s * 32, 16, 1024), tc::sdesc_sw128(b0 + s * 32, 16, 1024),
+                             idesc, s > 0);
             tc::mma_commit(bar);
         }
-        if (!mma_wait()) goto cleanup;
+        if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
-        // row i of A = [M | R_f C | R_b C]
+        // row r of A: half g of M (columns 64g .. 64g+63), then R_f C (g = 0) or R_b C (g = 1)
         {
-            const uint32_t lane_base = (uint32_t)(warp * 32);
-            const float ff = __expf(ci - r);    // forward row factor
-            const float fb = __expf(r - ei);    // flipped row factor
-            for (int cc = 0; cc < 4; ++cc) {
+            const float ff = __expf(ci - rmid), fb = __expf(rmid - ei);
+            const int wq = warp & 3;  // this warp's rows are 32*wq .. 32*wq + 31
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int cc = 2 * g + half;  // 32-column chunk of S
                 float sv[32];
                 tc::tmem_ld32(tc::tmem_addr(tmem + kColS, lane_base, cc * 32), sv);
                 tc::tmem_wait_ld();
+                if (factored && cc < wq) {           // every column left of every row: forward only
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float m[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = cc * 32 + q * 8 + e;
-                        float w;
-                        if (factored) {
-                            w = (j <= i ? ff * sm.gf()[j] : 0.f) + (j >= i ? fb * sm.gb()[j] : 0.f);
-                        } else {
-                            const float cj = sm.cum()[k * kSub + j], dj = sm.dt()[k * kSub + j];
-                            const float ej = cj - dj * Ah;
-                            w = ((j <= i ? __expf(ci - cj) : 0.f) + (j >= i ? __expf(ej - ei) : 0.f)) * dj;
-                        }
-                        m[e] = sv[q * 8 + e] * w;
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 f = *reinterpret_cast<const float4 *>(sgf + cc * 32 + 4 * q);
+                        sv[4 * q] *= ff * f.x;
+                        sv[4 * q + 1] *= ff * f.y;
+                        sv[4 * q + 2] *= ff * f.z;
+                        sv[4 * q + 3] *= ff * f.w;
                     }
-                    const int j0 = cc * 32 + q * 8;
-                    put_chunk(sm.A(j0 >> 6), i, (j0 & 63) >> 3, m);
+                } else if (factored && cc > wq) {    // every column right of every row: flipped only
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 f = *reinterpret_cast<const float4 *>(sgb + cc * 32 + 4 * q);
+                        sv[4 * q] *= fb * f.x;
+                        sv[4 * q + 1] *= fb * f.y;
+                        sv[4 * q + 2] *= fb * f.z;
+                        sv[4 * q + 3] *= fb * f.w;
+                    }
+                } else if (factored) {               // the diagonal block
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        const int j = cc * 32 + q;
+                        const float w = (j <= r ? ff * sgf[j] : 0.f) + (j >= r ? fb * sgb[j] : 0.f);
+                        sv[q] *= w;
+                    }
+                } else {                             // decay range too wide: exact exponentials
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        const int j = cc * 32 + q;
+                        const float cj = scum[k * kSub + j], dj = sdt[k * kSub + j];
+                        const float ej = cj - dj * Ah;
+                        sv[q] *= ((j <= r ? __expf(ci - cj) : 0.f) + (j >= r ? __expf(ej - ei) : 0.f)) * dj;
+                    }
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) put_chunk(sA + g * kTile, r, half * 4 + q, sv + 8 * q);
             }
-            const float rf = __expf(ci), rb = __expf(cend - ei);
+            const float rs = g == 0 ? __expf(ci) : __expf(cend - ei);
+            uint8_t *dst = sA + (2 + g) * kTile;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                float v[8], vf[8], vb[8];
-                row_chunk(sm.C(buf), i, ch, v);
+                float v[8];
+                row_chunk(sC(buf), r, ch, v);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    vf[e] = rf * v[e];
-                    vb[e] = rb * v[e];
-                }
-                put_chunk(sm.A(2), i, ch, vf);
-                put_chunk(sm.A(3), i, ch, vb);
+                for (int u = 0; u < 8; ++u) v[u] *= rs;
+                put_chunk(dst, r, ch, v);
             }
         }
         tc::fence_proxy_async_smem();
@@ -398,8 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
             tc::tc_fence_after();
             const uint32_t id_mx = tc::idesc_bf16(128, 64, 0, 1);
             const uint32_t id_ch = tc::idesc_bf16(128, 64, 0, 0);
-            const uint32_t a0 = tc::smem_u32(sm.A(0)), x0 = tc::smem_u32(sm.X(buf));
-            const uint32_t hf = tc::smem_u32(sm.Hf()), hb = tc::smem_u32(sm.Hb());
+            const uint32_t a0 = tc::smem_u32(sA), x0 = tc::smem_u32(sX(buf));
+            const uint32_t hf = tc::smem_u32(sHf), hb = tc::smem_u32(sHb);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
                 tc::mma_bf16(tmem + kColAcc, tc::sdesc_sw128(a0 + (s >> 2) * kTile + (s & 3) * 32, 16, 1024),
@@ -414,33 +461,29 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
                              tc::sdesc_sw128(hb + s * 32, 16, 1024), id_ch, true);
             tc::mma_commit(bar);
         }
-        if (!mma_wait()) goto cleanup;
+        if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
-        // epilogue: y_i = Acc_i + 2 D x_i -> grid position of token i. The TMEM loads are
-        // warp-collective, so every lane issues them; only lanes of real tokens store.
+        // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r -> grid position of token r.
+        // The TMEM load is warp-collective: every lane issues it, only real tokens store.
         {
-            const uint32_t lane_base = (uint32_t)(warp * 32);
-            const bool valid = n < len;
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
-                                 (((size_t)b * a.N + (valid ? sm.goff()[n] : 0)) * a.nh + h) * 64;
-            for (int half = 0; half < 2; ++half) {
-                float acc[32];
-                tc::tmem_ld32(tc::tmem_addr(tmem + kColAcc, lane_base, half * 32), acc);
-                tc::tmem_wait_ld();
-                if (valid) {
+            float acc[32];
+            tc::tmem_ld32(tc::tmem_addr(tmem + kColAcc, lane_base, 32 * g), acc);
+            tc::tmem_wait_ld();
+            if (n < len) {
+                __nv_bfloat16 *dst =
+                    static_cast<__nv_bfloat16 *>(a.out) + (((size_t)b * a.N + sgoff[n]) * a.nh + h) * 64 + 32 * g;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float xv[8], y[8];
-                        row_chunk(sm.X(buf), i, half * 4 + q, xv);
+                for (int q = 0; q < 4; ++q) {
+                    float xv[8], y[8];
+                    row_chunk(sX(buf), r, 4 * g + q, xv);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = acc[q * 8 + e] + 2.f * Dh * xv[e];
-                        uint4 u;
-                        u.x = tc::pack_bf16(y[0], y[1]);
-                        u.y = tc::pack_bf16(y[2], y[3]);
-                        u.z = tc::pack_bf16(y[4], y[5]);
-                        u.w = tc::pack_bf16(y[6], y[7]);
-                        *reinterpret_cast<uint4 *>(dst + half * 32 + q * 8) = u;
-                    }
+                    for (int u = 0; u < 8; ++u) y[u] = fmaf(Dh2, xv[u], acc[8 * q + u]);
+                    uint4 o;
+                    o.x = tc::pack_bf16(y[0], y[1]);
+                    o.y = tc::pack_bf16(y[2], y[3]);
+                    o.z = tc::pack_bf16(y[4], y[5]);
+                    o.w = tc::pack_bf16(y[6], y[7]);
+                    *reinterpret_cast<uint4 *>(dst + 8 * q) = o;
                 }
             }
         }
@@ -459,12 +502,151 @@ cleanup:
     }
 }
 
+// ---------------------------------------------------------------------------
+// chunk_state
+// ---------------------------------------------------------------------------
+constexpr uint32_t kStOffX = 0;            // 2 buffers
+constexpr uint32_t kStOffB = 2 * kTile;    // 2 buffers
+constexpr uint32_t kStOffU = 4 * kTile;    // U_f, U_b
+constexpr uint32_t kStOffDt = 6 * kTile;
+constexpr uint32_t kStOffCum = kStOffDt + kMaxChunk * 4;
+constexpr uint32_t kStOffGoff = kStOffCum + kMaxChunk * 4;
+constexpr uint32_t kStOffRed = kStOffGoff + kMaxChunk * 4;  // 8 floats
+constexpr uint32_t kStOffBar = kStOffRed + 64;
+constexpr uint32_t kStSmemBytes = kStOffBar + 64 + 1024;
+
+__global__ void __launch_bounds__(kThreads, 2) ssd_chunk_state_tc_kernel(SsdArgs a, int nsub)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    auto tX = [base](int i) { return base + kStOffX + i * kTile; };
+    auto tB = [base](int i) { return base + kStOffB + i * kTile; };
+    uint8_t *uf = base + kStOffU, *ub = base + kStOffU + kTile;
+    float *sdt = reinterpret_cast<float *>(base + kStOffDt);
+    float *scum = reinterpret_cast<float *>(base + kStOffCum);
+    int *sgoff = reinterpret_cast<int *>(base + kStOffGoff);
+    float *sred = reinterpret_cast<float *>(base + kStOffRed);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + kStOffBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kStOffBar + 8);
+    int *abort_flag = reinterpret_cast<int *>(base + kStOffBar + 12);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int r = tid & (kSub - 1), g = tid >> 7;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
+    const int L = nsub * kSub;
+    const int n0 = c * L, len = min(L, a.N - n0);
+    const int grp = h / (a.nh / a.G);
+    const float Ah = a.A[h];
+    uint32_t mma_phase = 0;
+
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 64);
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::fence_mbar_init();
+        *abort_flag = 0;
+    }
+    load_chunk_meta(a, b, h, n0, len, L, sgoff, sdt);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    sub_cumsums(sdt, scum, Ah, nsub, true, sred);
+    const float cend = scum[L - 1];
+
+    load_rows(a, tX(0), tB(0), nullptr, sgoff, b, h, grp, len, 0);
+    for (int k = 0; k < nsub; ++k) {
+        const int buf = k & 1;
+        if (k + 1 < nsub) load_rows(a, tX(buf ^ 1), tB(buf ^ 1), nullptr, sgoff, b, h, grp, len, k + 1);
+        wait_loads(k + 1 < nsub);
+        __syncthreads();
+        {
+            const int n = k * kSub + r;
+            const float cj = scum[n], dj = sdt[n];
+            build_u(tX(buf), uf, ub, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
+        }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tc_fence_after();
+            mma_states(tmem, tc::smem_u32(uf), tc::smem_u32(tB(buf)), k > 0);
+            tc::mma_commit(bar);
+        }
+        if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto done;
+    }
+    {
+        // TMEM rows 0-63: forward state rows p, rows 64-127: flipped state rows p
+        const bool fwd = r < 64;
+        float *dst = (fwd ? a.states_f : a.states_b) + ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + (r & 63)) * 64 +
+                     32 * g;
+        float v[32];
+        tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, 32 * g), v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(dst + q * 4) = make_float4(v[q * 4], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+        if (tid == 0) a.alpha[((size_t)b * a.nh + h) * a.nchunks + c] = __expf(cend);
+    }
+done:
+    tc::cp_async_wait_all();
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 64);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// state_chain: one thread per element of the 64 x 64 state.
+// grid: (4096 / 256, nh * batch, 2 directions)
+// ---------------------------------------------------------------------------
+constexpr int kAhead = 8;
+
+__global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
+{
+    const int e = blockIdx.x * 256 + threadIdx.x;
+    const int hb = blockIdx.y, dir = blockIdx.z;
+    const int h = hb % a.nh, b = hb / a.nh;
+    const int nc = a.nchunks;
+    float *S = (dir == 0 ? a.states_f : a.states_b) + ((size_t)b * a.nh + h) * nc * 4096 + e;
+    const float *al = a.alpha + ((size_t)b * a.nh + h) * nc;
+    float hv = a.review ? a.h_init[((size_t)b * a.nh + h) * 4096 + e] : 0.f;
+    // visit chunks in chain order: forward 0 .. nc-1, flipped nc-1 .. 0
+    const int step = dir == 0 ? 1 : -1;
+    int cidx = dir == 0 ? 0 : nc - 1;
+    int left = nc;
+    while (left >= kAhead) {
+        float buf[kAhead], alp[kAhead];
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            buf[u] = S[(size_t)(cidx + u * step) * 4096];
+            alp[u] = al[cidx + u * step];
+        }
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            S[(size_t)(cidx + u * step) * 4096] = hv;
+            hv = fmaf(alp[u], hv, buf[u]);
+        }
+        cidx += kAhead * step;
+        left -= kAhead;
+    }
+    for (; left > 0; --left, cidx += step) {
+        const float v = S[(size_t)cidx * 4096];
+        S[(size_t)cidx * 4096] = hv;
+        hv = fmaf(al[cidx], hv, v);
+    }
+}
+
 }  // namespace
 
 bool ssd_tc_supported(const SsdArgs &a)
 {
     return a.bf16 && a.P == 64 && a.Ns == 64 && a.dirs == MATE_DIR_BI && a.Q % kSub == 0 && a.Q / kSub >= 1 &&
-           a.Q / kSub <= kMaxSubs && a.nchunks <= 65535 && a.nh <= 65535 && a.batch <= 65535;
+           a.Q / kSub <= kMaxSubs && a.nchunks <= 65535 && a.nh <= 65535 && a.batch <= 65535 &&
+           (size_t)a.nh * a.batch <= 65535;
 }
 
 cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
@@ -472,10 +654,26 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(ssd_chunk_out_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = launch_ssd_prepass_bf16_64(a, s);
+    e = cudaFuncSetAttribute(ssd_chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kStSmemBytes);
     if (e != cudaSuccess) return e;
-    Phase ph(MATE_PHASE_CHUNK_OUT, s);
-    ssd_chunk_out_tc_kernel<<<dim3(a.nh, a.nchunks, a.batch), kThreads, kSmemBytes, s>>>(a, a.Q / kSub);
+    if (a.review) {
+        e = launch_review_bf16_64(a, s);
+        if (e != cudaSuccess) return e;
+    }
+    const int nsub = a.Q / kSub;
+    {
+        Phase ph(MATE_PHASE_CHUNK_STATE, s);
+        ssd_chunk_state_tc_kernel<<<dim3(a.nh, a.nchunks, a.batch), kThreads, kStSmemBytes, s>>>(a, nsub);
+    }
+    {
+        Phase ph(MATE_PHASE_STATE_PASS, s);
+        ssd_state_chain_kernel<<<dim3(4096 / 256, a.nh * a.batch, 2), 256, 0, s>>>(a);
+    }
+    {
+        Phase ph(MATE_PHASE_CHUNK_OUT, s);
+        ssd_chunk_out_tc_kernel<<<dim3(a.nh, a.nchunks, a.batch), kThreads, kSmemBytes, s>>>(a, nsub);
+    }
     return cudaGetLastError();
 }
 

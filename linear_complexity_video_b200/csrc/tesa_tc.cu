@@ -38,7 +38,7 @@ namespace {
 constexpr int kThreads = 128;
 constexpr uint32_t kTile = 16384;  // one 128-row x 128-byte box
 constexpr uint32_t kSmemData = 6 * kTile;
-constexpr uint32_t kSmemBytes = kSmemData + 1024 /*alignment slack*/ + 64;
+constexpr uint32_t kSmemBytes = kSmemData + 1024 /*alignment slack*/ + 64;  // + barriers, flags, key mask
 
 struct TesaTcParams {
     int T, H, W, nh;
@@ -98,12 +98,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int tt = t0 + r / ss, hh = h0 + (r / p.Sw) % p.Sw, ww = w0 + r % p.Sw;
         return tt >= 0 && tt < p.T && hh >= 0 && hh < p.H && ww >= 0 && ww < p.W;
     };
-    uint32_t kmask[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t m = 0;
-        for (int j = 0; j < 32; ++j) m |= (uint32_t)row_valid(c * 32 + j) << j;
-        kmask[c] = m;
+    // key validity mask: thread r evaluates row r once, warp ballots share it
+    uint32_t *smask = reinterpret_cast<uint32_t *>(abort_flag + 1);
+    const bool qvalid = row_valid(tid);
+    {
+        const uint32_t m = __ballot_sync(0xffffffffu, qvalid);
+        if ((tid & 31) == 0) smask[warp] = m;
     }
 
     if (!tc::mbar_wait(bar_load, 0, p.err)) atomicExch(abort_flag, 1);
@@ -112,6 +112,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::mbar_wait(bar_load, 0, nullptr);  // bounded second chance for copies in flight
         goto cleanup;
     }
+    uint32_t kmask[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) kmask[c] = smask[c];
 
     // ---- S = Q K^T --------------------------------------------------------
     if (tid == 0) {
@@ -197,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::tc_fence_after();
 
         // ---- epilogue: row tid of O / sum -> global --------------------------
-        const bool qvalid = row_valid(tid);
         const int tt = t0 + tid / ss, hh = h0 + (tid / p.Sw) % p.Sw, ww = w0 + tid % p.Sw;
         __nv_bfloat16 *dst =
             qvalid ? p.out + ((((size_t)tt * p.H + hh) * p.W + ww) * p.nh + head) * 128 : nullptr;
