@@ -25,14 +25,16 @@ struct SsdArgs {
     int review;              // 1 when a review prefix precedes the scan
     int pt, ph, pw;          // review pooling box
     int Tp, Hp, Wp, Np;      // pooled grid and its token count
+    int pool_splits;         // each pooling box is summed in this many parts
     int bf16;                // 1: x, B, C, out are bf16; 0: fp32
     // workspace carve-outs (fp32)
     float *states_f;         // (batch, nh, nchunks, P, Ns): chunk-local forward states,
-                             //   overwritten by the state entering each chunk
+                             //   overwritten by the state entering each chunk (the
+                             //   tensor-core path stores them as bf16)
     float *states_b;         // same for the flipped scan
     float *alpha;            // (batch, nh, nchunks): exp(A * sum of dt over the chunk)
     float *h_init;           // (batch, nh, P, Ns): state after the review prefix
-    float *pooled;           // (batch, Np, nh*P + nh + G*Ns): pooled x, dt, B
+    float *pooled;           // (batch, pool_splits, Np, nh*P + nh + G*Ns): partial box sums of x, dt, B
     int *err;                // device error word (MATE_ERR_* set by bounded waits)
 };
 

@@ -107,6 +107,14 @@ int ssd_shape(int T, int H, int W, const int *pool, const mate_ssd_dims *d, int 
         a.Hp = H / pool[1];
         a.Wp = W / pool[2];
         a.Np = a.Tp * a.Hp * a.Wp;
+        // split each pooling box so that the pooling grid covers the GPU a few times over
+        const int64_t box = (int64_t)a.pt * a.ph * a.pw;
+        const int64_t blocks = (int64_t)a.Np * a.batch * ((a.nh * a.P + a.nh + a.G * a.Ns) / 8 / 256 + 1);
+        int64_t splits = (1184 + blocks - 1) / blocks;
+        if (splits > 8) splits = 8;
+        if (splits > box) splits = box;
+        if (splits < 1) splits = 1;
+        a.pool_splits = (int)splits;
     }
     return MATE_OK;
 }
@@ -182,7 +190,8 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a)
     if (a.review) off = align_up(off + (size_t)a.batch * a.nh * a.P * a.Ns * sizeof(float));
     l.pooled = off;
     if (a.review)
-        off = align_up(off + (size_t)a.batch * a.Np * ((size_t)a.nh * a.P + a.nh + (size_t)a.G * a.Ns) * sizeof(float));
+        off = align_up(off + (size_t)a.batch * a.pool_splits * a.Np *
+                                 ((size_t)a.nh * a.P + a.nh + (size_t)a.G * a.Ns) * sizeof(float));
     l.total = off;
     return l;
 }

@@ -39,13 +39,20 @@ constexpr int kMaxStateChunk = 1024;  // chunk_state handles chunks of up to thi
 __device__ __forceinline__ size_t tok_index(const SsdArgs &a, int b, int g) { return (size_t)b * a.N + g; }
 
 // ---------------------------------------------------------------------------
-// review_pool: pooled[b][cell][ch] = mean over the cell's box of x | dt | B
-// grid: (Np, ceil(channels / 256), batch)
+// review_pool: pooled[b][s][cell][ch] = sum of x | dt | B over part s of the
+// cell's box (the box's tokens, row-major, cut into pool_splits ranges).
+// grid: (Np, ceil(channels / 256), batch * pool_splits)
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void split_range(int box, int splits, int s, int &lo, int &hi)
+{
+    lo = (int)(((long long)box * s) / splits);
+    hi = (int)(((long long)box * (s + 1)) / splits);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) review_pool_kernel(SsdArgs a)
 {
-    const int cell = blockIdx.x, b = blockIdx.z;
+    const int cell = blockIdx.x, b = blockIdx.z / a.pool_splits, sp = blockIdx.z % a.pool_splits;
     const int CX = a.nh * a.P, CD = a.nh, CB = a.G * a.Ns, CH = CX + CD + CB;
     const int ch = blockIdx.y * blockDim.x + threadIdx.x;
     if (ch >= CH) return;
@@ -53,20 +60,21 @@ __global__ void __launch_bounds__(kThreads) review_pool_kernel(SsdArgs a)
     const int tp = cell / hw, r = cell - tp * hw, hp = r / a.Wp, wp = r - hp * a.Wp;
     const T *x = static_cast<const T *>(a.x);
     const T *Bm = static_cast<const T *>(a.B);
+    int lo, hi;
+    split_range(a.pt * a.ph * a.pw, a.pool_splits, sp, lo, hi);
     float sum = 0.f;
-    for (int i = 0; i < a.pt; ++i)
-        for (int j = 0; j < a.ph; ++j)
-            for (int k = 0; k < a.pw; ++k) {
-                const int g = ((tp * a.pt + i) * a.H + hp * a.ph + j) * a.W + wp * a.pw + k;
-                const size_t tok = tok_index(a, b, g);
-                if (ch < CX)
-                    sum += ld(x + tok * CX + ch);
-                else if (ch < CX + CD)
-                    sum += a.dt[tok * CD + (ch - CX)];
-                else
-                    sum += ld(Bm + tok * CB + (ch - CX - CD));
-            }
-    a.pooled[((size_t)b * a.Np + cell) * CH + ch] = sum / (float)(a.pt * a.ph * a.pw);
+    for (int q = lo; q < hi; ++q) {
+        const int i = q / (a.ph * a.pw), rr = q - i * (a.ph * a.pw), j = rr / a.pw, k = rr - j * a.pw;
+        const int g = ((tp * a.pt + i) * a.H + hp * a.ph + j) * a.W + wp * a.pw + k;
+        const size_t tok = tok_index(a, b, g);
+        if (ch < CX)
+            sum += ld(x + tok * CX + ch);
+        else if (ch < CX + CD)
+            sum += a.dt[tok * CD + (ch - CX)];
+        else
+            sum += ld(Bm + tok * CB + (ch - CX - CD));
+    }
+    a.pooled[(((size_t)b * a.pool_splits + sp) * a.Np + cell) * CH + ch] = sum;
 }
 
 // ---------------------------------------------------------------------------
@@ -78,25 +86,26 @@ __global__ void __launch_bounds__(kThreads) review_pool_kernel(SsdArgs a)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
 {
-    const int cell = blockIdx.x, b = blockIdx.z;
+    const int cell = blockIdx.x, b = blockIdx.z / a.pool_splits, sp = blockIdx.z % a.pool_splits;
     const int CX = a.nh * a.P, CD = a.nh, CB = a.G * a.Ns, CH = CX + CD + CB;
     const int VX = CX / 8, VB = CB / 8, VD = CD / 4;
     const int v = blockIdx.y * blockDim.x + threadIdx.x;
     if (v >= VX + VB + VD) return;
     const int hw = a.Hp * a.Wp;
     const int tp = cell / hw, r = cell - tp * hw, hp = r / a.Wp, wp = r - hp * a.Wp;
-    const int box = a.pt * a.ph * a.pw;
+    int lo, hi;
+    split_range(a.pt * a.ph * a.pw, a.pool_splits, sp, lo, hi);
     const int kind = v < VX ? 0 : (v < VX + VB ? 1 : 2);
     float acc[4][8];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
-    for (int i0 = 0; i0 < box; i0 += 4) {
+    for (int i0 = lo; i0 < hi; i0 += 4) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = i0 + u;
-            if (i >= box) break;
+            if (i >= hi) break;
             const int it = i / (a.ph * a.pw), rr = i - it * (a.ph * a.pw), ih = rr / a.pw, iw = rr - ih * a.pw;
             const int g = ((tp * a.pt + it) * a.H + hp * a.ph + ih) * a.W + wp * a.pw + iw;
             const size_t tok = (size_t)b * a.N + g;
@@ -120,11 +129,10 @@ __global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
             }
         }
     }
-    const float inv = 1.f / (float)box;
     float out[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * inv;
-    float *dst = a.pooled + ((size_t)b * a.Np + cell) * CH;
+    for (int e = 0; e < 8; ++e) out[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
+    float *dst = a.pooled + (((size_t)b * a.pool_splits + sp) * a.Np + cell) * CH;
     if (kind == 0) {
         dst += v * 8;
     } else if (kind == 1) {
@@ -153,6 +161,7 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
     const int CX = a.nh * a.P, CD = a.nh, CH = CX + CD + a.G * a.Ns;
     const float Ah = a.A[h];
     const int L = 2 * a.Np;
+    const float inv_box = 1.f / (float)(a.pt * a.ph * a.pw);
     float s[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) s[e] = 0.f;
@@ -164,13 +173,17 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
             if (pos >= L) continue;
             const int r = pos < a.Np ? pos : L - 1 - pos;  // [R, flip(R)]
             const int cell = rms_grid_offset(r, a.Tp, a.Hp, a.Wp, a.mode);
-            const float *row = a.pooled + ((size_t)b * a.Np + cell) * CH;
+            const int col = c < P ? h * P + c : (c < P + NS ? CX + CD + grp * NS + (c - P) : CX + h);
+            float v = 0.f;
+            for (int sp = 0; sp < a.pool_splits; ++sp)
+                v += a.pooled[(((size_t)b * a.pool_splits + sp) * a.Np + cell) * CH + col];
+            v *= inv_box;
             if (c < P)
-                xs[k][c] = row[h * P + c];
+                xs[k][c] = v;
             else if (c < P + NS)
-                bs[k][c - P] = row[CX + CD + grp * NS + (c - P)];
+                bs[k][c - P] = v;
             else
-                ds[k] = row[CX + h];
+                ds[k] = v;
         }
         __syncthreads();
         const int kmax = min(kTile, L - base);
@@ -409,7 +422,7 @@ cudaError_t run_prepass(const SsdArgs &a, cudaStream_t s)
         const int CH = a.nh * a.P + a.nh + a.G * a.Ns;
         {
             Phase ph(MATE_PHASE_REVIEW_POOL, s);
-            review_pool_kernel<T><<<dim3(a.Np, (CH + kThreads - 1) / kThreads, a.batch), kThreads, 0, s>>>(a);
+            review_pool_kernel<T><<<dim3(a.Np, (CH + kThreads - 1) / kThreads, a.batch * a.pool_splits), kThreads, 0, s>>>(a);
         }
         {
             Phase ph(MATE_PHASE_REVIEW_SCAN, s);
@@ -471,9 +484,11 @@ cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)
         Phase ph(MATE_PHASE_REVIEW_POOL, s);
         if (vec) {
             const int nv = a.nh * a.P / 8 + a.G * a.Ns / 8 + a.nh / 4;
-            review_pool_vec_kernel<<<dim3(a.Np, (nv + kThreads - 1) / kThreads, a.batch), kThreads, 0, s>>>(a);
+            review_pool_vec_kernel<<<dim3(a.Np, (nv + kThreads - 1) / kThreads, a.batch * a.pool_splits), kThreads, 0,
+                                     s>>>(a);
         } else {
-            review_pool_kernel<__nv_bfloat16><<<dim3(a.Np, (CH + kThreads - 1) / kThreads, a.batch), kThreads, 0, s>>>(a);
+            review_pool_kernel<__nv_bfloat16>
+                <<<dim3(a.Np, (CH + kThreads - 1) / kThreads, a.batch * a.pool_splits), kThreads, 0, s>>>(a);
         }
     }
     {

@@ -18,7 +18,9 @@
 //              chunk); rows 0-63 forward, rows 64-127 flipped.
 // state_chain  one thread per state element replaces every chunk-local state
 //              by the state entering the chunk (forward from the left, flipped
-//              from the right), starting from the review state or zero.
+//              from the right), starting from the review state or zero. The
+//              chunk states are stored as bf16 (halving their traffic); the
+//              chain accumulates in fp32.
 // chunk_out    phase 1: the same MMA per sub-chunk with sub-chunk-local
 //              weights, each result kept in its own TMEM slot;
 //              phase 2: chain the slots in TMEM from the chunk's entering
@@ -306,16 +308,19 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
     {
         const bool fwd = r < 64;
         const int p = fwd ? r : r - 64;
-        const float *Hin =
-            (fwd ? a.states_f : a.states_b) + ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + p) * 64 + 32 * g;
+        const __nv_bfloat16 *Hin = reinterpret_cast<const __nv_bfloat16 *>(fwd ? a.states_f : a.states_b) +
+                                   ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + p) * 64 + 32 * g;
         float hv[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 v = *reinterpret_cast<const float4 *>(Hin + 4 * q);
-            hv[4 * q] = v.x;
-            hv[4 * q + 1] = v.y;
-            hv[4 * q + 2] = v.z;
-            hv[4 * q + 3] = v.w;
+        for (int q = 0; q < 4; ++q) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(Hin + 8 * q);
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = tc::unpack_bf16(w4[e]);
+                hv[8 * q + 2 * e] = f.x;
+                hv[8 * q + 2 * e + 1] = f.y;
+            }
         }
         for (int it = 0; it < nsub; ++it) {
             const int k = fwd ? it : nsub - 1 - it;
@@ -503,26 +508,26 @@ cleanup:
 }
 
 // ---------------------------------------------------------------------------
-// chunk_state
+// chunk_state: ~54 KB of shared memory and 64 TMEM columns, so four CTAs
+// share an SM and their loads overlap each other's math. U_f is written over
+// the x tile it is computed from.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kStOffX = 0;            // 2 buffers
-constexpr uint32_t kStOffB = 2 * kTile;    // 2 buffers
-constexpr uint32_t kStOffU = 4 * kTile;    // U_f, U_b
-constexpr uint32_t kStOffDt = 6 * kTile;
+constexpr uint32_t kStOffX = 0;            // x, then U_f
+constexpr uint32_t kStOffU = kTile;        // U_b (right after U_f: the MMA's second M group)
+constexpr uint32_t kStOffB = 2 * kTile;
+constexpr uint32_t kStOffDt = 3 * kTile;
 constexpr uint32_t kStOffCum = kStOffDt + kMaxChunk * 4;
 constexpr uint32_t kStOffGoff = kStOffCum + kMaxChunk * 4;
 constexpr uint32_t kStOffRed = kStOffGoff + kMaxChunk * 4;  // 8 floats
 constexpr uint32_t kStOffBar = kStOffRed + 64;
 constexpr uint32_t kStSmemBytes = kStOffBar + 64 + 1024;
 
-__global__ void __launch_bounds__(kThreads, 2) ssd_chunk_state_tc_kernel(SsdArgs a, int nsub)
+__global__ void __launch_bounds__(kThreads, 4) ssd_chunk_state_tc_kernel(SsdArgs a, int nsub)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    auto tX = [base](int i) { return base + kStOffX + i * kTile; };
-    auto tB = [base](int i) { return base + kStOffB + i * kTile; };
-    uint8_t *uf = base + kStOffU, *ub = base + kStOffU + kTile;
+    uint8_t *tX = base + kStOffX, *tB = base + kStOffB, *ub = base + kStOffU;
     float *sdt = reinterpret_cast<float *>(base + kStOffDt);
     float *scum = reinterpret_cast<float *>(base + kStOffCum);
     int *sgoff = reinterpret_cast<int *>(base + kStOffGoff);
@@ -555,38 +560,42 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_state_tc_kernel(SsdArgs
     sub_cumsums(sdt, scum, Ah, nsub, true, sred);
     const float cend = scum[L - 1];
 
-    load_rows(a, tX(0), tB(0), nullptr, sgoff, b, h, grp, len, 0);
     for (int k = 0; k < nsub; ++k) {
-        const int buf = k & 1;
-        if (k + 1 < nsub) load_rows(a, tX(buf ^ 1), tB(buf ^ 1), nullptr, sgoff, b, h, grp, len, k + 1);
-        wait_loads(k + 1 < nsub);
+        load_rows(a, tX, tB, nullptr, sgoff, b, h, grp, len, k);
+        wait_loads(false);
         __syncthreads();
         {
             const int n = k * kSub + r;
             const float cj = scum[n], dj = sdt[n];
-            build_u(tX(buf), uf, ub, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
+            build_u(tX, tX, ub, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc::tc_fence_after();
-            mma_states(tmem, tc::smem_u32(uf), tc::smem_u32(tB(buf)), k > 0);
+            mma_states(tmem, tc::smem_u32(tX), tc::smem_u32(tB), k > 0);
             tc::mma_commit(bar);
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto done;
     }
     {
-        // TMEM rows 0-63: forward state rows p, rows 64-127: flipped state rows p
+        // TMEM rows 0-63: forward state rows p, rows 64-127: flipped state rows p (stored as bf16)
         const bool fwd = r < 64;
-        float *dst = (fwd ? a.states_f : a.states_b) + ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + (r & 63)) * 64 +
-                     32 * g;
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(fwd ? a.states_f : a.states_b) +
+                             ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + (r & 63)) * 64 + 32 * g;
         float v[32];
         tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, 32 * g), v);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4 *>(dst + q * 4) = make_float4(v[q * 4], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+        for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = tc::pack_bf16(v[8 * q], v[8 * q + 1]);
+            o.y = tc::pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+            o.z = tc::pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+            o.w = tc::pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+            *reinterpret_cast<uint4 *>(dst + 8 * q) = o;
+        }
         if (tid == 0) a.alpha[((size_t)b * a.nh + h) * a.nchunks + c] = __expf(cend);
     }
 done:
@@ -600,7 +609,8 @@ done:
 }
 
 // ---------------------------------------------------------------------------
-// state_chain: one thread per element of the 64 x 64 state.
+// state_chain: one thread per element of the 64 x 64 state. The chunk states
+// are stored as bf16; the chain itself runs in fp32.
 // grid: (4096 / 256, nh * batch, 2 directions)
 // ---------------------------------------------------------------------------
 constexpr int kAhead = 8;
@@ -611,7 +621,8 @@ __global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
     const int hb = blockIdx.y, dir = blockIdx.z;
     const int h = hb % a.nh, b = hb / a.nh;
     const int nc = a.nchunks;
-    float *S = (dir == 0 ? a.states_f : a.states_b) + ((size_t)b * a.nh + h) * nc * 4096 + e;
+    __nv_bfloat16 *S = reinterpret_cast<__nv_bfloat16 *>(dir == 0 ? a.states_f : a.states_b) +
+                       ((size_t)b * a.nh + h) * nc * 4096 + e;
     const float *al = a.alpha + ((size_t)b * a.nh + h) * nc;
     float hv = a.review ? a.h_init[((size_t)b * a.nh + h) * 4096 + e] : 0.f;
     // visit chunks in chain order: forward 0 .. nc-1, flipped nc-1 .. 0
@@ -622,20 +633,20 @@ __global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
         float buf[kAhead], alp[kAhead];
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) {
-            buf[u] = S[(size_t)(cidx + u * step) * 4096];
+            buf[u] = __bfloat162float(S[(size_t)(cidx + u * step) * 4096]);
             alp[u] = al[cidx + u * step];
         }
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) {
-            S[(size_t)(cidx + u * step) * 4096] = hv;
+            S[(size_t)(cidx + u * step) * 4096] = __float2bfloat16_rn(hv);
             hv = fmaf(alp[u], hv, buf[u]);
         }
         cidx += kAhead * step;
         left -= kAhead;
     }
     for (; left > 0; --left, cidx += step) {
-        const float v = S[(size_t)cidx * 4096];
-        S[(size_t)cidx * 4096] = hv;
+        const float v = __bfloat162float(S[(size_t)cidx * 4096]);
+        S[(size_t)cidx * 4096] = __float2bfloat16_rn(hv);
         hv = fmaf(al[cidx], hv, v);
     }
 }

@@ -6,9 +6,11 @@
 // shifted on alternate layers, with partial windows at both ends of a shifted
 // axis.
 //
-// One CTA of 128 threads per (window, head); two CTAs fit on an SM (96 KB of
-// shared memory and 256 TMEM columns each), so one CTA's loads overlap the
-// other's math.
+// One persistent CTA per SM walks (window, head) items with two shared-memory
+// stages and two TMEM buffers, so the loads of one item, the tensor-core work
+// of another and the softmax of a third overlap: a producer warp issues the
+// TMA loads, an MMA warp issues tcgen05.mma, and two warpgroups take turns
+// with the softmax and the epilogue.
 //   1. TMA loads the window's Q, K, V boxes (64 head-dims x Sw x Sw x Tw each,
 //      two per tensor) straight from the (T, H, W, heads, d) layout. The box
 //      origin is the window's first grid coordinate, possibly negative for a
@@ -35,45 +37,91 @@ namespace mate {
 
 namespace {
 
-constexpr int kThreads = 128;
-constexpr uint32_t kTile = 16384;  // one 128-row x 128-byte box
-constexpr uint32_t kSmemData = 6 * kTile;
-constexpr uint32_t kSmemBytes = kSmemData + 1024 /*alignment slack*/ + 64;  // + barriers, flags, key mask
+constexpr uint32_t kTile = 16384;           // one 128-row x 128-byte box
+constexpr uint32_t kStage = 6 * kTile;      // Q (2 tiles, later P), K (2), V (2)
+constexpr int kStages = 2;
+constexpr int kWG = 128;                    // a softmax / epilogue warpgroup
+constexpr int kProducerWarp = 8;            // TMA loads
+constexpr int kMmaWarp = 9;                 // tcgen05.mma issue
+constexpr int kThreads = 320;               // warpgroups 0 and 1 (warps 0-7), producer, MMA
+constexpr uint32_t kSmemBytes = kStages * kStage + 1024 /*alignment slack*/ + 256;
 
 struct TesaTcParams {
     int T, H, W, nh;
     int Tw, Sw;
     int offt, offh, offw;
     int nwh, nww;
+    int items;          // windows * heads
     float scale_log2;   // log2(e) / sqrt(d)
     __nv_bfloat16 *out; // batch element base
     int *err;
 };
 
-__global__ void __launch_bounds__(kThreads, 2)
+struct Item {
+    int head, t0, h0, w0;
+};
+
+// Items are ordered (window, head) with heads fastest and dealt round-robin:
+// CTA c takes c, c + G, c + 2G, ... (G CTAs), so at any moment the CTAs work
+// on neighbouring windows and share DRAM rows and L2 lines.
+__device__ __forceinline__ Item item_of(const TesaTcParams &p, int local)
+{
+    const int item = blockIdx.x + local * gridDim.x;
+    Item it;
+    it.head = item % p.nh;
+    const int wid = item / p.nh;
+    const int kw = wid % p.nww, kh = (wid / p.nww) % p.nwh, kt = wid / (p.nww * p.nwh);
+    it.t0 = kt * p.Tw - p.offt;
+    it.h0 = kh * p.Sw - p.offh;
+    it.w0 = kw * p.Sw - p.offw;
+    return it;
+}
+
+// is box row r (r = (tt*Sw + hh)*Sw + ww) inside the grid?
+__device__ __forceinline__ bool row_in_grid(const TesaTcParams &p, const Item &it, int r)
+{
+    const int ss = p.Sw * p.Sw;
+    const int tt = it.t0 + r / ss, hh = it.h0 + (r / p.Sw) % p.Sw, ww = it.w0 + r % p.Sw;
+    return tt >= 0 && tt < p.T && hh >= 0 && hh < p.H && ww >= 0 && ww < p.W;
+}
+
+// Persistent CTA (one per SM) walking its share of the items; its i-th item
+// uses smem stage i % 2 and TMEM buffers S[i % 2], O[i % 2].
+//   producer warp : TMA Q, K, V of item i into its stage once the stage is free
+//   MMA warp      : S = Q K^T once loaded (and the TMEM buffer is free);
+//                   O = P V once the warpgroup has written P
+//   warpgroups    : warpgroup g takes the items with i % 2 == g: softmax into
+//                   P, then (after P V) the epilogue
+__global__ void __launch_bounds__(kThreads, 1)
     tesa_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, TesaTcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    uint8_t *sQ = smem;              // 2 tiles; later holds P
-    uint8_t *sK = smem + 2 * kTile;  // 2 tiles
-    uint8_t *sV = smem + 4 * kTile;  // 2 tiles
-    uint64_t *bar_load = reinterpret_cast<uint64_t *>(smem + kSmemData);
-    uint64_t *bar_mma = bar_load + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 2);
-    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStage);
+    uint64_t *full = bars;         // [2] stage loaded
+    uint64_t *empty = bars + 2;    // [2] stage consumed (P V done)
+    uint64_t *s_full = bars + 4;   // [2] S in TMEM
+    uint64_t *p_full = bars + 6;   // [2] P written (128 arrivals)
+    uint64_t *o_full = bars + 8;   // [2] O in TMEM
+    uint64_t *t_empty = bars + 10; // [2] O read out (128 arrivals)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int head = blockIdx.x, wid = blockIdx.y;  // heads fastest: they share DRAM rows
-    const int kw = wid % p.nww, kh = (wid / p.nww) % p.nwh, kt = wid / (p.nww * p.nwh);
-    const int t0 = kt * p.Tw - p.offt, h0 = kh * p.Sw - p.offh, w0 = kw * p.Sw - p.offw;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_items = p.items > (int)blockIdx.x ? (p.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
-    if (warp == 0) tc::tmem_alloc(tmem_slot, 256);
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
     if (tid == 0) {
-        tc::mbar_init(bar_load, 1);
-        tc::mbar_init(bar_mma, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&full[i], 1);
+            tc::mbar_init(&empty[i], 1);
+            tc::mbar_init(&s_full[i], 1);
+            tc::mbar_init(&p_full[i], kWG);
+            tc::mbar_init(&o_full[i], 1);
+            tc::mbar_init(&t_empty[i], kWG);
+        }
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
@@ -81,153 +129,171 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
 
-    if (tid == 0) {
-        tc::mbar_expect_tx(bar_load, 6 * kTile);
-        for (int half = 0; half < 2; ++half) {
-            tc::tma_load_5d(sQ + half * kTile, &mq, bar_load, half * 64, head, w0, h0, t0);
-            tc::tma_load_5d(sK + half * kTile, &mk, bar_load, half * 64, head, w0, h0, t0);
-            tc::tma_load_5d(sV + half * kTile, &mv, bar_load, half * 64, head, w0, h0, t0);
-        }
-    }
-
-    // which of the 128 box rows are inside the grid (row r = (tt*Sw + hh)*Sw + ww)
-    const int ss = p.Sw * p.Sw;
-    auto row_valid = [&](int r) {
-        const int tt = t0 + r / ss, hh = h0 + (r / p.Sw) % p.Sw, ww = w0 + r % p.Sw;
-        return tt >= 0 && tt < p.T && hh >= 0 && hh < p.H && ww >= 0 && ww < p.W;
+    // Waits inside a role are made warp-uniform, so a warp leaves its loop as a
+    // whole and every thread reaches the final __syncthreads.
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, tc::mbar_wait_or_abort(bar, parity, p.err, abort_flag)) != 0;
     };
-    // key validity mask: thread r evaluates row r once, warp ballots share it
-    uint32_t *smask = reinterpret_cast<uint32_t *>(abort_flag + 1);
-    const bool qvalid = row_valid(tid);
-    {
-        const uint32_t m = __ballot_sync(0xffffffffu, qvalid);
-        if ((tid & 31) == 0) smask[warp] = m;
-    }
-
-    if (!tc::mbar_wait(bar_load, 0, p.err)) atomicExch(abort_flag, 1);
-    __syncthreads();
-    if (*abort_flag) {
-        tc::mbar_wait(bar_load, 0, nullptr);  // bounded second chance for copies in flight
-        goto cleanup;
-    }
-    uint32_t kmask[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) kmask[c] = smask[c];
-
-    // ---- S = Q K^T --------------------------------------------------------
-    if (tid == 0) {
-        tc::tc_fence_after();
-        const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 0);
-        const uint32_t q0 = tc::smem_u32(sQ), k0 = tc::smem_u32(sK);
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            const uint32_t off = (s >> 2) * kTile + (s & 3) * 32;
-            tc::mma_bf16(tS, tc::sdesc_sw128(q0 + off, 16, 1024), tc::sdesc_sw128(k0 + off, 16, 1024), idesc, s > 0);
-        }
-        tc::mma_commit(bar_mma);
-    }
-    if (!tc::mbar_wait(bar_mma, 0, p.err)) atomicExch(abort_flag, 1);
-    __syncthreads();
-    if (*abort_flag) {
-        tc::mbar_wait(bar_mma, 0, nullptr);
-        goto cleanup;
-    }
-    tc::tc_fence_after();
-
-    // ---- softmax of row tid -> P (bf16, K-major swizzled, into sQ) ---------
-    {
-        const uint32_t lane_base = (uint32_t)(warp * 32);
-        float s[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), s[c]);
-        tc::tmem_wait_ld();
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if ((kmask[c] >> j) & 1u) mx = fmaxf(mx, s[c][j]);
-        const float mxs = mx * p.scale_log2;
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float e = ((kmask[c] >> j) & 1u) ? exp2f(fmaf(s[c][j], p.scale_log2, -mxs)) : 0.f;
-                s[c][j] = e;
-                sum += e;
-            }
-        // row tid of P: keys 0..63 in tile 0, 64..127 in tile 1; 8 keys per 16-byte chunk
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int key0 = c * 32 + q * 8;
-                uint4 v;
-                v.x = tc::pack_bf16(s[c][q * 8 + 0], s[c][q * 8 + 1]);
-                v.y = tc::pack_bf16(s[c][q * 8 + 2], s[c][q * 8 + 3]);
-                v.z = tc::pack_bf16(s[c][q * 8 + 4], s[c][q * 8 + 5]);
-                v.w = tc::pack_bf16(s[c][q * 8 + 6], s[c][q * 8 + 7]);
-                uint8_t *tile = sQ + (key0 >> 6) * kTile;
-                *reinterpret_cast<uint4 *>(tile + tc::sw128(tid, (key0 & 63) >> 3)) = v;
-            }
-        const float inv = 1.f / sum;
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // ---- O = P V ---------------------------------------------------------
-        if (tid == 0) {
-            tc::tc_fence_after();
-            const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
-            const uint32_t p0 = tc::smem_u32(sQ), v0 = tc::smem_u32(sV);
-#pragma unroll
-            for (int st = 0; st < 8; ++st) {
-                const uint32_t aoff = (st >> 2) * kTile + (st & 3) * 32;
-                tc::mma_bf16(tO, tc::sdesc_sw128(p0 + aoff, 16, 1024), tc::sdesc_sw128(v0 + st * 2048, kTile, 1024),
-                             idesc, st > 0);
-            }
-            tc::mma_commit(bar_mma);
-        }
-        if (!tc::mbar_wait(bar_mma, 1, p.err)) atomicExch(abort_flag, 1);
-        __syncthreads();
-        if (*abort_flag) {
-            tc::mbar_wait(bar_mma, 1, nullptr);
-            goto cleanup;
-        }
-        tc::tc_fence_after();
-
-        // ---- epilogue: row tid of O / sum -> global --------------------------
-        const int tt = t0 + tid / ss, hh = h0 + (tid / p.Sw) % p.Sw, ww = w0 + tid % p.Sw;
-        __nv_bfloat16 *dst =
-            qvalid ? p.out + ((((size_t)tt * p.H + hh) * p.W + ww) * p.nh + head) * 128 : nullptr;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tc::tmem_ld32(tc::tmem_addr(tO, lane_base, c * 32), o);
-            tc::tmem_wait_ld();
-            if (qvalid) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 v;
-                    v.x = tc::pack_bf16(o[q * 8 + 0] * inv, o[q * 8 + 1] * inv);
-                    v.y = tc::pack_bf16(o[q * 8 + 2] * inv, o[q * 8 + 3] * inv);
-                    v.z = tc::pack_bf16(o[q * 8 + 4] * inv, o[q * 8 + 5] * inv);
-                    v.w = tc::pack_bf16(o[q * 8 + 6] * inv, o[q * 8 + 7] * inv);
-                    *reinterpret_cast<uint4 *>(dst + c * 32 + q * 8) = v;
+    if (warp == kProducerWarp) {
+        for (int i = 0; i < n_items; ++i) {
+            const int s = i & 1;
+            if (i >= 2 && !wait_all(&empty[s], ((i >> 1) - 1) & 1)) break;
+            if (lane == 0) {
+                const Item it = item_of(p, i);
+                uint8_t *st = smem + s * kStage;
+                tc::mbar_expect_tx(&full[s], kStage);
+                for (int half = 0; half < 2; ++half) {
+                    tc::tma_load_5d(st + half * kTile, &mq, &full[s], half * 64, it.head, it.w0, it.h0, it.t0);
+                    tc::tma_load_5d(st + (2 + half) * kTile, &mk, &full[s], half * 64, it.head, it.w0, it.h0, it.t0);
+                    tc::tma_load_5d(st + (4 + half) * kTile, &mv, &full[s], half * 64, it.head, it.w0, it.h0, it.t0);
                 }
             }
+            __syncwarp();
+        }
+    } else if (warp == kMmaWarp) {
+        // S(i+1) is issued before waiting for P(i), so both warpgroups stay busy
+        const uint32_t id_s = tc::idesc_bf16(128, 128, 0, 0);
+        const uint32_t id_o = tc::idesc_bf16(128, 128, 0, 1);
+        auto issue_s = [&](int i) -> bool {
+            const int s = i & 1;
+            const uint32_t ph = (i >> 1) & 1;
+            if (!wait_all(&full[s], ph)) return false;
+            if (i >= 2 && !wait_all(&t_empty[s], ph ^ 1)) return false;
+            tc::tc_fence_after();
+            if (lane == 0) {
+                const uint32_t q0 = tc::smem_u32(smem + s * kStage), k0 = q0 + 2 * kTile;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k >> 2) * kTile + (k & 3) * 32;
+                    tc::mma_bf16(tmem + s * 256, tc::sdesc_sw128(q0 + off, 16, 1024), tc::sdesc_sw128(k0 + off, 16, 1024),
+                                 id_s, k > 0);
+                }
+                tc::mma_commit(&s_full[s]);
+            }
+            __syncwarp();
+            return true;
+        };
+        if (n_items > 0 && issue_s(0)) {
+            for (int i = 0; i < n_items; ++i) {
+                if (i + 1 < n_items && !issue_s(i + 1)) break;
+                const int s = i & 1;
+                if (!wait_all(&p_full[s], (i >> 1) & 1)) break;
+                tc::tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t p0 = tc::smem_u32(smem + s * kStage), v0 = p0 + 4 * kTile;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t aoff = (k >> 2) * kTile + (k & 3) * 32;
+                        tc::mma_bf16(tmem + s * 256 + 128, tc::sdesc_sw128(p0 + aoff, 16, 1024),
+                                     tc::sdesc_sw128(v0 + k * 2048, kTile, 1024), id_o, k > 0);
+                    }
+                    tc::mma_commit(&o_full[s]);
+                    tc::mma_commit(&empty[s]);
+                }
+                __syncwarp();
+            }
+        }
+    } else {
+        // ---- warpgroup g handles the items i with i % 2 == g (stage and TMEM buffer g)
+        const int g = warp >> 2, row = tid & (kWG - 1);
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        const uint32_t tS = tmem + g * 256, tO = tS + 128;
+        for (int i = g; i < n_items; i += 2) {
+            const uint32_t ph = (i >> 1) & 1;
+            const Item it = item_of(p, i);
+            // key validity: each warp ballots all 128 rows itself
+            uint32_t kmask[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) kmask[c] = __ballot_sync(0xffffffffu, row_in_grid(p, it, c * 32 + lane));
+            if (!wait_all(&s_full[g], ph)) break;
+            tc::tc_fence_after();
+            // pass 1: row maximum over the keys in the grid
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float sv[32];
+                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if ((kmask[c] >> j) & 1u) mx = fmaxf(mx, sv[j]);
+            }
+            // pass 2: P = exp(S - max) as bf16 into the stage's Q tiles, and the row sum
+            const float mxs = mx * p.scale_log2;
+            float sum = 0.f;
+            uint8_t *pq = smem + g * kStage;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float sv[32];
+                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float e = ((kmask[c] >> j) & 1u) ? exp2f(fmaf(sv[j], p.scale_log2, -mxs)) : 0.f;
+                    sv[j] = e;
+                    sum += e;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int key0 = c * 32 + q * 8;
+                    uint4 v;
+                    v.x = tc::pack_bf16(sv[q * 8 + 0], sv[q * 8 + 1]);
+                    v.y = tc::pack_bf16(sv[q * 8 + 2], sv[q * 8 + 3]);
+                    v.z = tc::pack_bf16(sv[q * 8 + 4], sv[q * 8 + 5]);
+                    v.w = tc::pack_bf16(sv[q * 8 + 6], sv[q * 8 + 7]);
+                    *reinterpret_cast<uint4 *>(pq + (key0 >> 6) * kTile + tc::sw128(row, (key0 & 63) >> 3)) = v;
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&p_full[g]);
+            const float inv = 1.f / sum;
+
+            // epilogue: O row / sum -> global, once P V is done
+            if (!wait_all(&o_full[g], ph)) break;
+            tc::tc_fence_after();
+            const bool qvalid = row_in_grid(p, it, row);
+            const int ss = p.Sw * p.Sw;
+            const int tt = it.t0 + row / ss, hh = it.h0 + (row / p.Sw) % p.Sw, ww = it.w0 + row % p.Sw;
+            __nv_bfloat16 *dst =
+                qvalid ? p.out + ((((size_t)tt * p.H + hh) * p.W + ww) * p.nh + it.head) * 128 : nullptr;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float o[32];
+                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, c * 32), o);
+                tc::tmem_wait_ld();
+                if (qvalid) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 v;
+                        v.x = tc::pack_bf16(o[q * 8 + 0] * inv, o[q * 8 + 1] * inv);
+                        v.y = tc::pack_bf16(o[q * 8 + 2] * inv, o[q * 8 + 3] * inv);
+                        v.z = tc::pack_bf16(o[q * 8 + 4] * inv, o[q * 8 + 5] * inv);
+                        v.w = tc::pack_bf16(o[q * 8 + 6] * inv, o[q * 8 + 7] * inv);
+                        *reinterpret_cast<uint4 *>(dst + c * 32 + q * 8) = v;
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            tc::mbar_arrive(&t_empty[g]);
         }
     }
 
-cleanup:
+    // all roles done (or aborted): make sure no MMA still writes TMEM, then free it
     tc::tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        // an aborted pipeline may still have copies or MMAs in flight: give them a
+        // bounded 200 us to land before the tensor memory is released
+        const uint64_t t0 = tc::globaltimer();
+        while (tc::globaltimer() - t0 < 200000ull) {
+        }
+    }
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, 256);
+        tc::tmem_dealloc(tmem, 512);
     }
 }
 
@@ -270,7 +336,7 @@ bool make_map(CUtensorMap *m, const void *base, const TesaArgs &a)
 bool tesa_tc_supported(const TesaArgs &a)
 {
     return a.bf16 && a.d == 128 && a.Tw * a.Sw * a.Sw == 128 && a.Sw <= 128 && a.Tw <= 128 &&
-           (size_t)a.nwt * a.nwh * a.nww <= 65535 &&
+           (size_t)a.nwt * a.nwh * a.nww * a.nh < ((size_t)1 << 31) &&
            encode_fn() != nullptr;
 }
 
@@ -294,6 +360,10 @@ cudaError_t launch_tesa_tc(const TesaArgs &a, cudaStream_t s)
     p.err = a.err;
     const size_t per_batch = (size_t)a.N * a.nh * 128;
     const int nwin = a.nwt * a.nwh * a.nww;
+    p.items = nwin * a.nh;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = p.items < sms ? p.items : sms;
     for (int b = 0; b < a.batch; ++b) {
         CUtensorMap mq, mk, mv;
         const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q) + b * per_batch;
@@ -302,7 +372,7 @@ cudaError_t launch_tesa_tc(const TesaArgs &a, cudaStream_t s)
         if (!make_map(&mq, q, a) || !make_map(&mk, k, a) || !make_map(&mv, v, a)) return cudaErrorInvalidValue;
         p.out = static_cast<__nv_bfloat16 *>(a.out) + b * per_batch;
         Phase ph(MATE_PHASE_TESA, s);
-        tesa_tc_kernel<<<dim3(a.nh, nwin), kThreads, kSmemBytes, s>>>(mq, mk, mv, p);
+        tesa_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
