@@ -218,14 +218,23 @@ __device__ __forceinline__ bool mma_wait(uint64_t *bar, uint32_t &phase, int *er
 }
 
 // ---------------------------------------------------------------------------
-// chunk_out
+// chunk_out: ~101 KB of shared memory, 256 TMEM columns and at most 128
+// registers per thread, so two CTAs share an SM.
+//   TMEM columns   0..127 : the K sub-chunk states, packed bf16 (32 columns each:
+//                           64 values of a state row per lane)
+//   TMEM columns 128..255 : phase 1 MMA result (64 cols), phase 3 S (128 cols),
+//                           then the output accumulator (64 cols)
+//   shared memory         : x, B, C tiles of one sub-chunk; two 16 KB tiles for
+//                           U_f / U_b (phase 1) or M (phase 3); h_f, h_b operands.
+//                           In phase 3, R_f C overwrites the C tile and R_b C the
+//                           B tile once S = C B^T is done.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kOffX = 0;                 // 2 buffers x 16 KB
-constexpr uint32_t kOffB = 2 * kTile;         // 2 buffers
-constexpr uint32_t kOffC = 4 * kTile;         // 2 buffers
-constexpr uint32_t kOffA = 6 * kTile;         // 4 tiles: phase 1 U_f, U_b; phase 3 M0, M1, R_f C, R_b C
-constexpr uint32_t kOffH = 10 * kTile;        // h_f (8 KB) then h_b (8 KB)
-constexpr uint32_t kOffDt = 11 * kTile;
+constexpr uint32_t kOffX = 0;
+constexpr uint32_t kOffB = kTile;
+constexpr uint32_t kOffC = 2 * kTile;
+constexpr uint32_t kOffM = 3 * kTile;       // 2 tiles: U_f, U_b / M0, M1
+constexpr uint32_t kOffH = 5 * kTile;       // h_f (8 KB) then h_b (8 KB)
+constexpr uint32_t kOffDt = 6 * kTile;
 constexpr uint32_t kOffCum = kOffDt + kMaxChunk * 4;
 constexpr uint32_t kOffGoff = kOffCum + kMaxChunk * 4;
 constexpr uint32_t kOffGf = kOffGoff + kMaxChunk * 4;
@@ -234,19 +243,17 @@ constexpr uint32_t kOffRed = kOffGb + kSub * 4;  // 8 floats
 constexpr uint32_t kOffBar = kOffRed + 64;
 constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;
 
-constexpr uint32_t kColS = kMaxSubs * 64;  // S (128 cols) after the state slots
-constexpr uint32_t kColAcc = kColS + 128;  // output accumulator (64 cols)
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColR = 128;   // scratch region after the packed state slots
+constexpr uint32_t kTmemCols = 256;
 
-__global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a, int nsub)
+__device__ __forceinline__ uint32_t bf2(float lo, float hi) { return tc::pack_bf16(lo, hi); }
+
+__global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a, int nsub)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    auto sX = [base](int i) { return base + kOffX + i * kTile; };
-    auto sB = [base](int i) { return base + kOffB + i * kTile; };
-    auto sC = [base](int i) { return base + kOffC + i * kTile; };
-    uint8_t *sA = base + kOffA;
+    uint8_t *sX = base + kOffX, *sB = base + kOffB, *sC = base + kOffC, *sM = base + kOffM;
     uint8_t *sHf = base + kOffH, *sHb = base + kOffH + 8192;
     float *sdt = reinterpret_cast<float *>(base + kOffDt);
     float *scum = reinterpret_cast<float *>(base + kOffCum);
@@ -279,32 +286,45 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const uint32_t tR = tmem + kColR;
     sub_cumsums(sdt, scum, Ah, nsub, false, sred);
 
-    // ---------------- phase 1: sub-chunk-local states -> TMEM slots ---------------
-    load_rows(a, sX(0), sB(0), nullptr, sgoff, b, h, grp, len, 0);
+    // ---------------- phase 1: sub-chunk-local states -> packed bf16 slots ------------
     for (int k = 0; k < nsub; ++k) {
-        const int buf = k & 1;
-        if (k + 1 < nsub) load_rows(a, sX(buf ^ 1), sB(buf ^ 1), nullptr, sgoff, b, h, grp, len, k + 1);
-        wait_loads(k + 1 < nsub);
+        load_rows(a, sX, sB, nullptr, sgoff, b, h, grp, len, k);
+        wait_loads(false);
         __syncthreads();
         {
             const int n = k * kSub + r;
             const float cj = scum[n], dj = sdt[n], cend = scum[k * kSub + kSub - 1];
-            build_u(sX(buf), sA, sA + kTile, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
+            build_u(sX, sM, sM + kTile, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc::tc_fence_after();
-            mma_states(tmem + k * 64, tc::smem_u32(sA), tc::smem_u32(sB(buf)), false);
+            mma_states(tR, tc::smem_u32(sM), tc::smem_u32(sB), false);
             tc::mma_commit(bar);
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
+        {
+            // fp32 result columns 32g .. 32g+31 of row r -> 16 packed columns of slot k
+            float v[32];
+            tc::tmem_ld32(tc::tmem_addr(tR, lane_base, 32 * g), v);
+            tc::tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk[q] = bf2(v[2 * q], v[2 * q + 1]);
+            tc::tmem_st16(tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g), pk);
+            tc::tmem_wait_st();
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
     }
 
-    // ---------------- phase 2: chain the sub-chunk states in TMEM ------------------
+    // ---------------- phase 2: chain the sub-chunk states ------------------------------
     {
         const bool fwd = r < 64;
         const int p = fwd ? r : r - 64;
@@ -325,14 +345,20 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
         for (int it = 0; it < nsub; ++it) {
             const int k = fwd ? it : nsub - 1 - it;
             const float alpha = __expf(scum[k * kSub + kSub - 1]);
-            const uint32_t ta = tc::tmem_addr(tmem, lane_base, k * 64 + 32 * g);
-            float t0[32];
-            tc::tmem_ld32(ta, t0);
+            const uint32_t ta = tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g);
+            uint32_t loc[16], pk[16];
+            tc::tmem_ld16(ta, loc);
             tc::tmem_wait_ld();
-            tc::tmem_st32(ta, hv);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk[q] = bf2(hv[2 * q], hv[2 * q + 1]);
+            tc::tmem_st16(ta, pk);
             tc::tmem_wait_st();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) hv[q] = fmaf(alpha, hv[q], t0[q]);
+            for (int q = 0; q < 16; ++q) {
+                const float2 f = tc::unpack_bf16(loc[q]);
+                hv[2 * q] = fmaf(alpha, hv[2 * q], f.x);
+                hv[2 * q + 1] = fmaf(alpha, hv[2 * q + 1], f.y);
+            }
         }
     }
     tc::tc_fence_before();
@@ -340,19 +366,19 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
     tc::tc_fence_after();
 
     // ---------------- phase 3: outputs ---------------------------------------------
-    load_rows(a, sX(0), sB(0), sC(0), sgoff, b, h, grp, len, 0);
     for (int k = 0; k < nsub; ++k) {
-        const int buf = k & 1;
-        if (k + 1 < nsub) load_rows(a, sX(buf ^ 1), sB(buf ^ 1), sC(buf ^ 1), sgoff, b, h, grp, len, k + 1);
-        // entering states of sub-chunk k -> bf16 operands (row r: forward if r < 64)
+        load_rows(a, sX, sB, sC, sgoff, b, h, grp, len, k);
+        // entering states of sub-chunk k (already bf16) -> operand rows (forward if r < 64)
         {
-            float t0[32];
-            tc::tmem_ld32(tc::tmem_addr(tmem, lane_base, k * 64 + 32 * g), t0);
+            uint32_t pk[16];
+            tc::tmem_ld16(tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g), pk);
             tc::tmem_wait_ld();
             uint8_t *ht = r < 64 ? sHf : sHb;
             const int p = r & 63;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) put_chunk(ht, p, 4 * g + q, t0 + 8 * q);
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(ht + tc::sw128(p, 4 * g + q)) =
+                    make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
         const int n = k * kSub + r;
         const float ci = scum[n], di = sdt[n];
@@ -365,130 +391,139 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_chunk_out_tc_kernel(SsdArgs a
         }
         const float range = block_max(g == 0 ? fmaxf(fabsf(ci - rmid), fabsf(ei - rmid)) : 0.f, sred);
         const bool factored = range <= kFactorLimit;
-        wait_loads(k + 1 < nsub);
+        wait_loads(false);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
 
-        // S = C B^T
+        // S = C B^T -> TMEM R
         if (tid == 0) {
             tc::tc_fence_after();
             const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 0);
-            const uint32_t c0 = tc::smem_u32(sC(buf)), b0 = tc::smem_u32(sB(buf));
+            const uint32_t c0 = tc::smem_u32(sC), b0 = tc::smem_u32(sB);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                tc::mma_bf16(tmem + kColS, tc::sdesc_sw128(c0 + s * 32, 16, 1024), tc::sdesc_sw128(b0 + s * 32, 16, 1024),
-                             idesc, s > 0);
+            for (int s2 = 0; s2 < 4; ++s2)
+                tc::mma_bf16(tR, tc::sdesc_sw128(c0 + s2 * 32, 16, 1024), tc::sdesc_sw128(b0 + s2 * 32, 16, 1024), idesc,
+                             s2 > 0);
             tc::mma_commit(bar);
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
-        // row r of A: half g of M (columns 64g .. 64g+63), then R_f C (g = 0) or R_b C (g = 1)
+        // row r of M: columns 64g .. 64g+63 of S times the decay factors -> tile g
         {
             const float ff = __expf(ci - rmid), fb = __expf(rmid - ei);
             const int wq = warp & 3;  // this warp's rows are 32*wq .. 32*wq + 31
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int cc = 2 * g + half;  // 32-column chunk of S
-                float sv[32];
-                tc::tmem_ld32(tc::tmem_addr(tmem + kColS, lane_base, cc * 32), sv);
+            for (int qq = 0; qq < 4; ++qq) {
+                const int j0 = 64 * g + 16 * qq;   // first of these 16 columns
+                uint32_t raw16[16];
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, j0), raw16);
                 tc::tmem_wait_ld();
-                if (factored && cc < wq) {           // every column left of every row: forward only
+                float sv[16];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 f = *reinterpret_cast<const float4 *>(sgf + cc * 32 + 4 * q);
-                        sv[4 * q] *= ff * f.x;
-                        sv[4 * q + 1] *= ff * f.y;
-                        sv[4 * q + 2] *= ff * f.z;
-                        sv[4 * q + 3] *= ff * f.w;
+                for (int e = 0; e < 16; ++e) sv[e] = __uint_as_float(raw16[e]);
+                const int cc = j0 >> 5;             // 32-column block of these columns
+                if (factored && cc < wq) {          // left of every row of this warp: forward only
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sv[e] *= ff * sgf[j0 + e];
+                } else if (factored && cc > wq) {   // right of every row: flipped only
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sv[e] *= fb * sgb[j0 + e];
+                } else if (factored) {              // the diagonal block
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = j0 + e;
+                        sv[e] *= (j <= r ? ff * sgf[j] : 0.f) + (j >= r ? fb * sgb[j] : 0.f);
                     }
-                } else if (factored && cc > wq) {    // every column right of every row: flipped only
+                } else {                            // decay range too wide: exact exponentials
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 f = *reinterpret_cast<const float4 *>(sgb + cc * 32 + 4 * q);
-                        sv[4 * q] *= fb * f.x;
-                        sv[4 * q + 1] *= fb * f.y;
-                        sv[4 * q + 2] *= fb * f.z;
-                        sv[4 * q + 3] *= fb * f.w;
-                    }
-                } else if (factored) {               // the diagonal block
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        const int j = cc * 32 + q;
-                        const float w = (j <= r ? ff * sgf[j] : 0.f) + (j >= r ? fb * sgb[j] : 0.f);
-                        sv[q] *= w;
-                    }
-                } else {                             // decay range too wide: exact exponentials
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        const int j = cc * 32 + q;
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = j0 + e;
                         const float cj = scum[k * kSub + j], dj = sdt[k * kSub + j];
                         const float ej = cj - dj * Ah;
-                        sv[q] *= ((j <= r ? __expf(ci - cj) : 0.f) + (j >= r ? __expf(ej - ei) : 0.f)) * dj;
+                        sv[e] *= ((j <= r ? __expf(ci - cj) : 0.f) + (j >= r ? __expf(ej - ei) : 0.f)) * dj;
                     }
                 }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) put_chunk(sA + g * kTile, r, half * 4 + q, sv + 8 * q);
+                uint8_t *tile = sM + g * kTile;
+                const int ch = (j0 & 63) >> 3;
+                *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch)) =
+                    make_uint4(bf2(sv[0], sv[1]), bf2(sv[2], sv[3]), bf2(sv[4], sv[5]), bf2(sv[6], sv[7]));
+                *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch + 1)) =
+                    make_uint4(bf2(sv[8], sv[9]), bf2(sv[10], sv[11]), bf2(sv[12], sv[13]), bf2(sv[14], sv[15]));
             }
+        }
+        {
+            // row r of C, scaled by R_f (g = 0, written over C) or R_b (g = 1, written over B)
             const float rs = g == 0 ? __expf(ci) : __expf(cend - ei);
-            uint8_t *dst = sA + (2 + g) * kTile;
+            uint4 cr[8];
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) cr[ch] = *reinterpret_cast<const uint4 *>(sC + tc::sw128(r, ch));
+            tc::tc_fence_before();
+            __syncthreads();  // every thread has its C row; S is consumed
+            uint8_t *dst = g == 0 ? sC : sB;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                float v[8];
-                row_chunk(sC(buf), r, ch, v);
+                const uint32_t w4[4] = {cr[ch].x, cr[ch].y, cr[ch].z, cr[ch].w};
+                uint32_t o4[4];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] *= rs;
-                put_chunk(dst, r, ch, v);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = tc::unpack_bf16(w4[e]);
+                    o4[e] = bf2(f.x * rs, f.y * rs);
+                }
+                *reinterpret_cast<uint4 *>(dst + tc::sw128(r, ch)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
 
-        // Acc = M x + (R_f C) h_f^T + (R_b C) h_b^T
+        // Acc = M x + (R_f C) h_f^T + (R_b C) h_b^T -> TMEM R columns 0..63
         if (tid == 0) {
             tc::tc_fence_after();
             const uint32_t id_mx = tc::idesc_bf16(128, 64, 0, 1);
             const uint32_t id_ch = tc::idesc_bf16(128, 64, 0, 0);
-            const uint32_t a0 = tc::smem_u32(sA), x0 = tc::smem_u32(sX(buf));
+            const uint32_t m0 = tc::smem_u32(sM), x0 = tc::smem_u32(sX);
+            const uint32_t cf = tc::smem_u32(sC), cb = tc::smem_u32(sB);
             const uint32_t hf = tc::smem_u32(sHf), hb = tc::smem_u32(sHb);
 #pragma unroll
-            for (int s = 0; s < 8; ++s)
-                tc::mma_bf16(tmem + kColAcc, tc::sdesc_sw128(a0 + (s >> 2) * kTile + (s & 3) * 32, 16, 1024),
-                             tc::sdesc_sw128(x0 + s * 2048, kTile, 1024), id_mx, s > 0);
+            for (int s2 = 0; s2 < 8; ++s2)
+                tc::mma_bf16(tR, tc::sdesc_sw128(m0 + (s2 >> 2) * kTile + (s2 & 3) * 32, 16, 1024),
+                             tc::sdesc_sw128(x0 + s2 * 2048, kTile, 1024), id_mx, s2 > 0);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                tc::mma_bf16(tmem + kColAcc, tc::sdesc_sw128(a0 + 2 * kTile + s * 32, 16, 1024),
-                             tc::sdesc_sw128(hf + s * 32, 16, 1024), id_ch, true);
+            for (int s2 = 0; s2 < 4; ++s2)
+                tc::mma_bf16(tR, tc::sdesc_sw128(cf + s2 * 32, 16, 1024), tc::sdesc_sw128(hf + s2 * 32, 16, 1024), id_ch,
+                             true);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                tc::mma_bf16(tmem + kColAcc, tc::sdesc_sw128(a0 + 3 * kTile + s * 32, 16, 1024),
-                             tc::sdesc_sw128(hb + s * 32, 16, 1024), id_ch, true);
+            for (int s2 = 0; s2 < 4; ++s2)
+                tc::mma_bf16(tR, tc::sdesc_sw128(cb + s2 * 32, 16, 1024), tc::sdesc_sw128(hb + s2 * 32, 16, 1024), id_ch,
+                             true);
             tc::mma_commit(bar);
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
         // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r -> grid position of token r.
-        // The TMEM load is warp-collective: every lane issues it, only real tokens store.
+        // TMEM loads are warp-collective: every lane issues them, only real tokens store.
         {
-            float acc[32];
-            tc::tmem_ld32(tc::tmem_addr(tmem + kColAcc, lane_base, 32 * g), acc);
-            tc::tmem_wait_ld();
-            if (n < len) {
-                __nv_bfloat16 *dst =
-                    static_cast<__nv_bfloat16 *>(a.out) + (((size_t)b * a.N + sgoff[n]) * a.nh + h) * 64 + 32 * g;
+            const bool valid = n < len;
+            __nv_bfloat16 *dst =
+                static_cast<__nv_bfloat16 *>(a.out) + (((size_t)b * a.N + (valid ? sgoff[n] : 0)) * a.nh + h) * 64 + 32 * g;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float xv[8], y[8];
-                    row_chunk(sX(buf), r, 4 * g + q, xv);
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t acc[16];
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g + 16 * hq), acc);
+                tc::tmem_wait_ld();
+                if (valid) {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) y[u] = fmaf(Dh2, xv[u], acc[8 * q + u]);
-                    uint4 o;
-                    o.x = tc::pack_bf16(y[0], y[1]);
-                    o.y = tc::pack_bf16(y[2], y[3]);
-                    o.z = tc::pack_bf16(y[4], y[5]);
-                    o.w = tc::pack_bf16(y[6], y[7]);
-                    *reinterpret_cast<uint4 *>(dst + 8 * q) = o;
+                    for (int q = 0; q < 2; ++q) {
+                        float xv[8];
+                        row_chunk(sX, r, 4 * g + 2 * hq + q, xv);
+                        uint32_t o4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            o4[e] = bf2(fmaf(Dh2, xv[2 * e], __uint_as_float(acc[8 * q + 2 * e])),
+                                        fmaf(Dh2, xv[2 * e + 1], __uint_as_float(acc[8 * q + 2 * e + 1])));
+                        *reinterpret_cast<uint4 *>(dst + 16 * hq + 8 * q) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                    }
                 }
             }
         }
