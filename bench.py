@@ -323,19 +323,132 @@ def run_mate(args, cfg, rank, world, dist):
     return result
 
 
+def time_config(cfg, mode, steps, warmup, seed=0):
+    """Device time (ms) of one step of cfg in scan order `mode`, plus per-phase ms."""
+    import torch
+
+    import linear_complexity_video_b200 as mate
+    from linear_complexity_video_b200 import _lib, api
+
+    stream = torch.cuda.current_stream()
+    d = {k: v.cuda() for k, v in workloads.generate(cfg, seed=seed).items()}
+    out_ssd = torch.empty_like(d["x"])
+    out_att = torch.empty_like(d["q"])
+    ws = api.bissd_workspace(d["x"], d["B"], cfg.review, cfg.chunk)
+    sdims = api.ssd_dims(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, cfg.ngroups, cfg.chunk, cfg.torch_dtype)
+    adims = api.attn_dims(cfg.batch, cfg.attn_heads, cfg.attn_dim, cfg.torch_dtype)
+
+    def step():
+        api.mate_bissd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], cfg.T, cfg.H, cfg.W, mode, cfg.review,
+                           out_ssd, sdims, ws, stream)
+        api.tesa_fwd(d["q"], d["k"], d["v"], cfg.T, cfg.H, cfg.W, cfg.Tw, cfg.Sw, cfg.shift, out_att, adims, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    marks = []
+
+    def hook(phase, is_end, strm, user):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        marks.append((phase, is_end, ev))
+
+    L = mate.load()
+    hook_c = _lib.PHASE_HOOK(hook)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    # one more pass with the phase hook for the per-kernel split
+    L.mate_set_phase_hook(hook_c, None)
+    step()
+    torch.cuda.synchronize()
+    L.mate_set_phase_hook(_lib.PHASE_HOOK(), None)
+    phases, opened = {}, {}
+    for ph, is_end, ev in marks:
+        if not is_end:
+            opened[ph] = ev
+        else:
+            phases[_lib.PHASES[ph]] = round(opened.pop(ph).elapsed_time(ev), 4)
+    if mate.mate_last_error() != 0:
+        raise RuntimeError("device error word set")
+    del d, out_ssd, out_att, ws
+    torch.cuda.empty_cache()
+    return ms, phases
+
+
+def run_report(args):
+    """Every bf16 grid in every scan order it lists, then the N sweep with a
+    linearity fit. One JSON line per measurement, then a summary line."""
+    import numpy as np
+    import torch
+
+    peaks, _ = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    for name, cfg in workloads.CONFIGS.items():
+        if cfg.dtype != "bf16":
+            continue
+        for mode in cfg.modes:
+            ms, phases = time_config(cfg, mode, args.steps, args.warmup)
+            per_tok = algorithmic_bytes(cfg)
+            path_bytes = (per_tok["bissd"] + per_tok["review_pool"] + per_tok["tesa"]) * cfg.tokens
+            print(json.dumps({"report": "config", "workload": name, "scan": workloads.MODE_NAMES[mode],
+                              "tokens": cfg.tokens, "ms_per_step": round(ms, 4),
+                              "mtokens_per_s": round(cfg.tokens / ms / 1e3, 3),
+                              "path_hbm_frac": round(path_bytes / (ms / 1e3) / 1e9 / hbm, 4),
+                              "phase_ms": phases}), flush=True)
+    Ns, ts = [], []
+    for cfg in workloads.sweep_configs():
+        ms, phases = time_config(cfg, cfg.modes[0], args.steps, args.warmup)
+        per_tok = algorithmic_bytes(cfg)
+        path_bytes = (per_tok["bissd"] + per_tok["review_pool"] + per_tok["tesa"]) * cfg.tokens
+        Ns.append(cfg.tokens)
+        ts.append(ms)
+        print(json.dumps({"report": "sweep", "workload": cfg.name, "tokens": cfg.tokens, "ms_per_step": round(ms, 4),
+                          "mtokens_per_s": round(cfg.tokens / ms / 1e3, 3),
+                          "path_hbm_frac": round(path_bytes / (ms / 1e3) / 1e9 / hbm, 4), "phase_ms": phases}),
+              flush=True)
+    N = np.array(Ns, dtype=np.float64)
+    t = np.array(ts, dtype=np.float64)
+    slope, icpt = np.polyfit(N, t, 1)
+    pred = slope * N + icpt
+    r2 = 1.0 - float(np.sum((t - pred) ** 2) / np.sum((t - t.mean()) ** 2))
+    rate = N / t / 1e3
+    big = rate[N >= 32768]
+    spread = float(np.max(np.abs(big / np.median(big) - 1.0))) if len(big) else None
+    print(json.dumps({"report": "linearity", "fit": "t_ms = a + b*N", "a_ms": round(float(icpt), 5),
+                      "b_ns_per_token": round(float(slope) * 1e6, 4), "r2": round(r2, 5),
+                      "max_rel_dev_mtokens_per_s_N_ge_32k": round(spread, 4) if spread is not None else None}),
+          flush=True)
+
+
 def load_traffic(kernel, cfg):
-    """DRAM bytes per launch of `kernel` from a committed ncu summary, if one
-    matches the current build and workload; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of `kernel` from profiles/traffic.txt, if a line
+    matches the workload and the kernel's source file is unchanged since the
+    capture; else None."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
-        with open(path) as f:
-            t = json.load(f)
-    except (OSError, ValueError):
+        lines = open(path).read().splitlines()
+    except OSError:
         return None
-    ent = t.get(kernel)
-    if not ent or ent.get("workload") != cfg.name:
-        return None
-    return ent.get("bytes_per_launch")
+    for ln in lines:
+        if not ln.strip() or ln.lstrip().startswith("#"):
+            continue
+        f = ln.split()
+        if len(f) < 5 or f[0] != kernel or f[1] != cfg.name:
+            continue
+        try:
+            sha = hashlib.sha1(open(os.path.join(ROOT, f[3]), "rb").read()).hexdigest()
+        except OSError:
+            return None
+        return int(f[2]) if sha == f[4] else None
+    return None
 
 
 def run_reference(args, cfg):
@@ -380,6 +493,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--chunk", type=int, default=0, help="override the scan chunk length (a tiling choice)")
+    ap.add_argument("--report", action="store_true",
+                    help="time every bf16 grid in each of its scan orders and the N sweep (one JSON line each)")
     ap.add_argument("--steps-ref", type=int, default=1)
     ap.add_argument("--warmup-ref", type=int, default=0)
     args = ap.parse_args()
@@ -394,6 +509,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, cfg)), flush=True)
+        return
+    if args.report:
+        run_report(args)
         return
 
     dist = None

@@ -96,14 +96,15 @@ __global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
     int lo, hi;
     split_range(a.pt * a.ph * a.pw, a.pool_splits, sp, lo, hi);
     const int kind = v < VX ? 0 : (v < VX + VB ? 1 : 2);
-    float acc[4][8];
+    constexpr int kU = 4;  // tokens in flight per thread (8 costs occupancy: more registers)
+    float acc[kU][8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < kU; ++u)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
-    for (int i0 = lo; i0 < hi; i0 += 4) {
+    for (int i0 = lo; i0 < hi; i0 += kU) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kU; ++u) {
             const int i = i0 + u;
             if (i >= hi) break;
             const int it = i / (a.ph * a.pw), rr = i - it * (a.ph * a.pw), ih = rr / a.pw, iw = rr - ih * a.pw;
@@ -146,17 +147,19 @@ __global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
 
 // ---------------------------------------------------------------------------
 // review_scan: h_init[b][h] = state after scanning [R, flip(R)] from zero,
-// R = pooled grid in scan order. grid: (nh, batch)
+// R = pooled grid in scan order. The P rows of the state evolve independently,
+// so RS CTAs split them. grid: (nh, batch, RS)
 // ---------------------------------------------------------------------------
-template <int P, int NS>
+template <int P, int NS, int RS>
 __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
 {
-    constexpr int PN = P * NS;
+    constexpr int PR = P / RS;  // state rows of this CTA
+    constexpr int PN = PR * NS;
     constexpr int E = (PN + kThreads - 1) / kThreads;
-    __shared__ float xs[kTile][P];
+    __shared__ float xs[kTile][PR];
     __shared__ float bs[kTile][NS];
     __shared__ float ds[kTile];
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int h = blockIdx.x, b = blockIdx.y, p0 = blockIdx.z * PR;
     const int grp = h / (a.nh / a.G);
     const int CX = a.nh * a.P, CD = a.nh, CH = CX + CD + a.G * a.Ns;
     const float Ah = a.A[h];
@@ -167,21 +170,21 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
     for (int e = 0; e < E; ++e) s[e] = 0.f;
     for (int base = 0; base < L; base += kTile) {
         __syncthreads();
-        for (int idx = threadIdx.x; idx < kTile * (P + NS + 1); idx += blockDim.x) {
-            const int k = idx / (P + NS + 1), c = idx - k * (P + NS + 1);
+        for (int idx = threadIdx.x; idx < kTile * (PR + NS + 1); idx += blockDim.x) {
+            const int k = idx / (PR + NS + 1), c = idx - k * (PR + NS + 1);
             const int pos = base + k;
             if (pos >= L) continue;
             const int r = pos < a.Np ? pos : L - 1 - pos;  // [R, flip(R)]
             const int cell = rms_grid_offset(r, a.Tp, a.Hp, a.Wp, a.mode);
-            const int col = c < P ? h * P + c : (c < P + NS ? CX + CD + grp * NS + (c - P) : CX + h);
+            const int col = c < PR ? h * P + p0 + c : (c < PR + NS ? CX + CD + grp * NS + (c - PR) : CX + h);
             float v = 0.f;
             for (int sp = 0; sp < a.pool_splits; ++sp)
                 v += a.pooled[(((size_t)b * a.pool_splits + sp) * a.Np + cell) * CH + col];
             v *= inv_box;
-            if (c < P)
+            if (c < PR)
                 xs[k][c] = v;
-            else if (c < P + NS)
-                bs[k][c - P] = v;
+            else if (c < PR + NS)
+                bs[k][c - PR] = v;
             else
                 ds[k] = v;
         }
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int idx = threadIdx.x + e * kThreads;
-        if (idx < PN) a.h_init[((size_t)b * a.nh + h) * PN + idx] = s[e];
+        if (idx < PN) a.h_init[((size_t)b * a.nh + h) * (P * NS) + p0 * NS + idx] = s[e];
     }
 }
 
@@ -426,7 +429,8 @@ cudaError_t run_prepass(const SsdArgs &a, cudaStream_t s)
         }
         {
             Phase ph(MATE_PHASE_REVIEW_SCAN, s);
-            review_scan_kernel<P, NS><<<dim3(a.nh, a.batch), kThreads, 0, s>>>(a);
+            constexpr int RS = P >= 32 ? P / 16 : 1;
+            review_scan_kernel<P, NS, RS><<<dim3(a.nh, a.batch, RS), kThreads, 0, s>>>(a);
         }
     }
     {
@@ -493,7 +497,7 @@ cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)
     }
     {
         Phase ph(MATE_PHASE_REVIEW_SCAN, s);
-        review_scan_kernel<64, 64><<<dim3(a.nh, a.batch), kThreads, 0, s>>>(a);
+        review_scan_kernel<64, 64, 4><<<dim3(a.nh, a.batch, 4), kThreads, 0, s>>>(a);
     }
     return cudaGetLastError();
 }

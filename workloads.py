@@ -23,6 +23,10 @@ either set can be drawn without the other):
     q, k, v ~ N(0, 1)
 Tensors the config marks bf16 (x, B, C, q, k, v) are cast to bf16 after the
 draw; dt, A and D stay fp32.
+
+`chunk` is the scan's tiling length, not part of the method: the output does
+not depend on it beyond rounding. The bf16 grids use 512-token chunks (the
+longest the tensor-core scan takes); the tiny fp32 case uses 32.
 """
 from __future__ import annotations
 
@@ -80,13 +84,13 @@ class Config:
 CONFIGS: Dict[str, Config] = {
     "tiny": Config("tiny", 1, 4, 8, 8, 2, 16, 16, 1, 32, "f32", (SR, SC, TR, TC), (2, 4, 4),
                    2, 16, 2, 4, (1, 2, 2)),
-    "256p-17s": Config("256p-17s", 1, 32, 16, 16, 80, 64, 64, 1, 256, "bf16", (SR,), None,
+    "256p-17s": Config("256p-17s", 1, 32, 16, 16, 80, 64, 64, 1, 512, "bf16", (SR,), None,
                        20, 128, 2, 8, (0, 0, 0)),
-    "512p-17s": Config("512p-17s", 1, 32, 32, 32, 80, 64, 64, 1, 256, "bf16", (SR, SC, TR, TC),
+    "512p-17s": Config("512p-17s", 1, 32, 32, 32, 80, 64, 64, 1, 512, "bf16", (SR, SC, TR, TC),
                        (4, 8, 8), 20, 128, 2, 8, (1, 4, 4)),
-    "512p-68s": Config("512p-68s", 1, 128, 32, 32, 80, 64, 64, 1, 256, "bf16", (TC,), (8, 8, 8),
+    "512p-68s": Config("512p-68s", 1, 128, 32, 32, 80, 64, 64, 1, 512, "bf16", (TC,), (8, 8, 8),
                        20, 128, 2, 8, (1, 4, 4)),
-    "768p-17s": Config("768p-17s", 2, 32, 48, 48, 80, 64, 64, 1, 256, "bf16", (SR, SC, TR, TC), None,
+    "768p-17s": Config("768p-17s", 2, 32, 48, 48, 80, 64, 64, 1, 512, "bf16", (SR, SC, TR, TC), None,
                        20, 128, 2, 8, (0, 0, 0)),
 }
 
