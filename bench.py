@@ -155,6 +155,30 @@ def oracle_sample(cfg, threads=None):
 
 
 # ---------------------------------------------------------------------------
+# multi-rank plumbing (weak scaling over independent grids, no data exchange)
+# ---------------------------------------------------------------------------
+def rank_seed(rank: int, base: int = 0) -> int:
+    """Each rank draws its own grid: seed = base + rank."""
+    return base + rank
+
+
+def max_over_ranks(ms: float, dist, device=None) -> float:
+    """The step time of the job is the slowest rank's (max all-reduce)."""
+    if dist is None:
+        return ms
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job Mtokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3) / 1e6
+
+
+# ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
 def run_mate(args, cfg, rank, world, dist):
@@ -171,7 +195,7 @@ def run_mate(args, cfg, rank, world, dist):
     stream = torch.cuda.current_stream()
     mode = cfg.modes[0]
 
-    host = workloads.generate(cfg, seed=rank)
+    host = workloads.generate(cfg, seed=rank_seed(rank))
     d = {k: v.to(dev) for k, v in host.items()}
     out_ssd = torch.empty_like(d["x"])
     out_att = torch.empty_like(d["q"])
@@ -228,12 +252,7 @@ def run_mate(args, cfg, rank, world, dist):
     launches = L.mate_kernel_launches() - launches0
     barrier()
     clocks = sampler.stop() if sampler else None
-    ms_total = ev0.elapsed_time(ev1)
-    t_local = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    ms_total = float(t_local.item())
-    ms_step = ms_total / args.steps
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / args.steps
 
     # per-phase average duration on this rank
     phase_ms = {}
@@ -273,10 +292,8 @@ def run_mate(args, cfg, rank, world, dist):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / k_e2e], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": cfg.tokens * world / (float(te.item()) / 1e3) / 1e6, "unit": "Mtokens/s",
+        te = max_over_ranks(e0.elapsed_time(e1) / k_e2e, dist, dev)
+        e2e = {"value": job_throughput(cfg.tokens, world, te), "unit": "Mtokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e}
 
     result = None
@@ -288,7 +305,7 @@ def run_mate(args, cfg, rank, world, dist):
         dom_bytes = per_tok.get(dom, 0) * cfg.tokens
         achieved = dom_bytes / (phase_avg[dom] / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
-        value = cfg.tokens * world / (ms_step / 1e3) / 1e6
+        value = job_throughput(cfg.tokens, world, ms_step)
         traffic = load_traffic(dom, cfg)
         result = {
             "metric": "MATE token-mix Mtokens/s on 1 B200 (bi-SSD+TESA)",
