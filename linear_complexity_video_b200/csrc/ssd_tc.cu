@@ -173,21 +173,26 @@ __device__ __forceinline__ void sub_cumsums(const float *dt, float *cum, float A
     }
 }
 
-// U_f row r = w_f[r] x_r and U_b row r = w_b[r] x_r for chunks [4g, 4g + 4)
+// U_f row r = w_f[r] x_r and U_b row r = w_b[r] x_r for chunks [4g, 4g + 4), as
+// packed bf16 products (w rounded to bf16 once; each product rounded once).
+__device__ __forceinline__ __nv_bfloat162 bf16x2_of(uint32_t u) { return *reinterpret_cast<__nv_bfloat162 *>(&u); }
+__device__ __forceinline__ uint32_t u32_of(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
+
+__device__ __forceinline__ uint4 scale_chunk(uint4 x, __nv_bfloat162 w)
+{
+    return make_uint4(u32_of(__hmul2(bf16x2_of(x.x), w)), u32_of(__hmul2(bf16x2_of(x.y), w)),
+                      u32_of(__hmul2(bf16x2_of(x.z), w)), u32_of(__hmul2(bf16x2_of(x.w), w)));
+}
+
 __device__ __forceinline__ void build_u(const uint8_t *tX, uint8_t *uf, uint8_t *ub, int r, int g, float wf, float wb)
 {
+    const __nv_bfloat162 f2 = __float2bfloat162_rn(wf), b2 = __float2bfloat162_rn(wb);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const int ch = 4 * g + q;
-        float v[8], f[8], e[8];
-        row_chunk(tX, r, ch, v);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            f[u] = wf * v[u];
-            e[u] = wb * v[u];
-        }
-        put_chunk(uf, r, ch, f);
-        put_chunk(ub, r, ch, e);
+        const uint32_t off = tc::sw128(r, 4 * g + q);
+        const uint4 x = *reinterpret_cast<const uint4 *>(tX + off);
+        *reinterpret_cast<uint4 *>(uf + off) = scale_chunk(x, f2);
+        *reinterpret_cast<uint4 *>(ub + off) = scale_chunk(x, b2);
     }
 }
 
@@ -423,12 +428,18 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
 #pragma unroll
                 for (int e = 0; e < 16; ++e) sv[e] = __uint_as_float(raw16[e]);
                 const int cc = j0 >> 5;             // 32-column block of these columns
-                if (factored && cc < wq) {          // left of every row of this warp: forward only
+                if (factored && cc != wq) {         // off the diagonal block: one direction only
+                    // left of every row of this warp: forward; right of every row: flipped
+                    const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? sgf : sgb) + j0);
+                    const float rf = cc < wq ? ff : fb;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) sv[e] *= ff * sgf[j0 + e];
-                } else if (factored && cc > wq) {   // right of every row: flipped only
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) sv[e] *= fb * sgb[j0 + e];
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 f4 = fac[q];
+                        sv[4 * q] *= rf * f4.x;
+                        sv[4 * q + 1] *= rf * f4.y;
+                        sv[4 * q + 2] *= rf * f4.z;
+                        sv[4 * q + 3] *= rf * f4.w;
+                    }
                 } else if (factored) {              // the diagonal block
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -454,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
         }
         {
             // row r of C, scaled by R_f (g = 0, written over C) or R_b (g = 1, written over B)
-            const float rs = g == 0 ? __expf(ci) : __expf(cend - ei);
+            const __nv_bfloat162 rs = __float2bfloat162_rn(g == 0 ? __expf(ci) : __expf(cend - ei));
             uint4 cr[8];
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) cr[ch] = *reinterpret_cast<const uint4 *>(sC + tc::sw128(r, ch));
@@ -462,16 +473,7 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             __syncthreads();  // every thread has its C row; S is consumed
             uint8_t *dst = g == 0 ? sC : sB;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint32_t w4[4] = {cr[ch].x, cr[ch].y, cr[ch].z, cr[ch].w};
-                uint32_t o4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = tc::unpack_bf16(w4[e]);
-                    o4[e] = bf2(f.x * rs, f.y * rs);
-                }
-                *reinterpret_cast<uint4 *>(dst + tc::sw128(r, ch)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-            }
+            for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(dst + tc::sw128(r, ch)) = scale_chunk(cr[ch], rs);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
