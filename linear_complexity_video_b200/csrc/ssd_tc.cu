@@ -61,26 +61,31 @@ constexpr float kFactorLimit = 80.f;  // |exponent| bound for the factored exps
 // Gather the 128 token rows of sub-chunk `sub` into swizzled tiles (x: the 64
 // head dims of head h; B and C: the 64 state dims of the head's group; tC may
 // be null). goff[n] is the grid offset of chunk position n; rows past the
-// sequence end are zero.
+// sequence end are zero. Eight consecutive threads copy the eight 16-byte
+// chunks of one row, so a warp reads four whole 128-byte rows.
 __device__ __forceinline__ void load_rows(const SsdArgs &a, uint8_t *tX, uint8_t *tB, uint8_t *tC, const int *goff,
                                           int b, int h, int grp, int len, int sub)
 {
-    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
-    const __nv_bfloat16 *Bm = static_cast<const __nv_bfloat16 *>(a.B);
-    const __nv_bfloat16 *Cm = static_cast<const __nv_bfloat16 *>(a.C);
-    const int ntiles = tC ? 3 : 2;
-    for (int idx = threadIdx.x; idx < ntiles * kSub * 8; idx += kThreads) {
-        const int tile = idx / (kSub * 8);
-        const int r = (idx >> 3) & (kSub - 1), c = idx & 7;
+    const int c = threadIdx.x & 7;
+    const char *xb = static_cast<const char *>(a.x) + ((size_t)h * 64 + c * 8) * 2;
+    const size_t gb = ((size_t)grp * 64 + c * 8) * 2;
+    const char *bb = static_cast<const char *>(a.B) + gb;
+    const char *cb = static_cast<const char *>(a.C) + gb;
+#pragma unroll
+    for (int q = 0; q < kSub / (kThreads / 8); ++q) {
+        const int r = (threadIdx.x >> 3) + q * (kThreads / 8);
         const int n = sub * kSub + r;
-        uint8_t *dst = (tile == 0 ? tX : tile == 1 ? tB : tC) + tc::sw128(r, c);
+        const uint32_t off = tc::sw128(r, c);
         if (n < len) {
             const size_t tok = (size_t)b * a.N + goff[n];
-            const __nv_bfloat16 *src = tile == 0 ? x + (tok * a.nh + h) * 64 + c * 8
-                                                 : (tile == 1 ? Bm : Cm) + (tok * a.G + grp) * 64 + c * 8;
-            tc::cp_async16(dst, src);
+            tc::cp_async16(tX + off, xb + tok * (size_t)a.nh * 128);
+            tc::cp_async16(tB + off, bb + tok * (size_t)a.G * 128);
+            if (tC) tc::cp_async16(tC + off, cb + tok * (size_t)a.G * 128);
         } else {
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(tX + off) = z;
+            *reinterpret_cast<uint4 *>(tB + off) = z;
+            if (tC) *reinterpret_cast<uint4 *>(tC + off) = z;
         }
     }
     tc::cp_async_commit();
@@ -206,16 +211,21 @@ __device__ __forceinline__ void mma_states(uint32_t d_tmem, uint32_t uf_addr, ui
                      tc::sdesc_sw128(b_addr + s * 2048, kTile, 1024), idesc, accumulate || s > 0);
 }
 
-// Bounded wait for the next MMA completion on `bar`; on timeout every thread
-// returns false (after a second bounded wait for the MMAs in flight).
+// Bounded wait for the next MMA completion on `bar`: warp 0 polls the barrier
+// while the other warps wait at __syncthreads (no issue slots spent). On
+// timeout every thread returns false, after a second bounded wait for the MMAs
+// in flight.
 __device__ __forceinline__ bool mma_wait(uint64_t *bar, uint32_t &phase, int *err, int *abort_flag)
 {
-    const bool ok = tc::mbar_wait(bar, phase & 1u, err);
+    if ((threadIdx.x >> 5) == 0) {
+        const bool ok = tc::mbar_wait(bar, phase & 1u, err);
+        if (!ok && threadIdx.x == 0) *abort_flag = 1;
+    }
     ++phase;
-    if (!ok) atomicExch(abort_flag, 1);
     __syncthreads();
     if (*abort_flag) {
-        tc::mbar_wait(bar, (phase - 1) & 1u, nullptr);
+        if (threadIdx.x == 0) tc::mbar_wait(bar, (phase - 1) & 1u, nullptr);
+        __syncthreads();
         return false;
     }
     tc::tc_fence_after();
