@@ -6,11 +6,13 @@
 // shifted on alternate layers, with partial windows at both ends of a shifted
 // axis.
 //
-// One persistent CTA per SM walks (window, head) items with two shared-memory
-// stages and two TMEM buffers, so the loads of one item, the tensor-core work
-// of another and the softmax of a third overlap: a producer warp issues the
-// TMA loads, an MMA warp issues tcgen05.mma, and two warpgroups take turns
-// with the softmax and the epilogue.
+// One persistent CTA per SM walks (window, head) items. Q and K of an item sit
+// in one of two shared-memory slots that are released as soon as S = Q K^T is
+// done; V sits in one of three slots released after O = P V; P goes to TMEM
+// over S (the A operand of P V is read from TMEM). Two warps issue the TMA
+// loads (Q+K and V), one warp issues tcgen05.mma, and two warpgroups take
+// turns with the softmax and the epilogue, so loads, tensor-core work and
+// softmax of neighbouring items overlap.
 //   1. TMA loads the window's Q, K, V boxes (64 head-dims x Sw x Sw x Tw each,
 //      two per tensor) straight from the (T, H, W, heads, d) layout. The box
 //      origin is the window's first grid coordinate, possibly negative for a
@@ -18,9 +20,8 @@
 //      entirely in these coordinates.
 //   2. S = Q K^T (M = N = K = 128) into TMEM.
 //   3. Thread i owns query i: it reads S row i from TMEM, masks keys outside
-//      the grid, and writes P = exp(S - max) as bf16 into shared memory
-//      (reusing Q's buffer) in the swizzled K-major operand layout.
-//   4. O = P V (V as an MN-major operand) into TMEM.
+//      the grid, and writes P = exp(S - max) as bf16 pairs back into TMEM.
+//   4. O = P V (P from TMEM, V as an MN-major shared-memory operand) into TMEM.
 //   5. Thread i scales O row i by 1 / sum(P) and stores it if query i is in
 //      the grid.
 // A window holds exactly one 128-token tile, so the softmax needs no online
@@ -38,13 +39,18 @@ namespace mate {
 namespace {
 
 constexpr uint32_t kTile = 16384;           // one 128-row x 128-byte box
-constexpr uint32_t kStage = 6 * kTile;      // Q (2 tiles, later P), K (2), V (2)
-constexpr int kStages = 2;
+constexpr int kQkSlots = 2;                 // Q + K of an item (4 tiles), free once S = Q K^T is done
+constexpr int kVSlots = 3;                  // V of an item (2 tiles), free once O = P V is done
+constexpr uint32_t kQkSlot = 4 * kTile;
+constexpr uint32_t kVSlot = 2 * kTile;
+constexpr uint32_t kOffV = kQkSlots * kQkSlot;
+constexpr uint32_t kOffBar = kOffV + kVSlots * kVSlot;
 constexpr int kWG = 128;                    // a softmax / epilogue warpgroup
-constexpr int kProducerWarp = 8;            // TMA loads
-constexpr int kMmaWarp = 9;                 // tcgen05.mma issue
-constexpr int kThreads = 320;               // warpgroups 0 and 1 (warps 0-7), producer, MMA
-constexpr uint32_t kSmemBytes = kStages * kStage + 1024 /*alignment slack*/ + 256;
+constexpr int kQkWarp = 8;                  // TMA loads of Q and K
+constexpr int kVWarp = 9;                   // TMA loads of V
+constexpr int kMmaWarp = 10;                // tcgen05.mma issue
+constexpr int kThreads = 352;               // warpgroups 0 and 1 (warps 0-7) + 3 single warps
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024 /*alignment slack*/;
 
 struct TesaTcParams {
     int T, H, W, nh;
@@ -85,13 +91,14 @@ __device__ __forceinline__ bool row_in_grid(const TesaTcParams &p, const Item &i
     return tt >= 0 && tt < p.T && hh >= 0 && hh < p.H && ww >= 0 && ww < p.W;
 }
 
-// Persistent CTA (one per SM) walking its share of the items; its i-th item
-// uses smem stage i % 2 and TMEM buffers S[i % 2], O[i % 2].
-//   producer warp : TMA Q, K, V of item i into its stage once the stage is free
-//   MMA warp      : S = Q K^T once loaded (and the TMEM buffer is free);
-//                   O = P V once the warpgroup has written P
-//   warpgroups    : warpgroup g takes the items with i % 2 == g: softmax into
-//                   P, then (after P V) the epilogue
+// Persistent CTA (one per SM) walking its share of the items.
+//   QK warp   : TMA Q and K of item i into QK slot i % 2 once S of item i-2 is done
+//   V warp    : TMA V of item i into V slot i % 3 once P V of item i-3 is done
+//   MMA warp  : S(i) = Q K^T into TMEM buffer i % 2 (once that buffer's previous
+//               item has been read out), then, one item behind, O = P V with P
+//               taken from TMEM (it overwrites S)
+//   warpgroup g takes items i % 2 == g: softmax of S into P (bf16, in TMEM),
+//               then the epilogue O / rowsum -> global
 __global__ void __launch_bounds__(kThreads, 1)
     tesa_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, TesaTcParams p)
@@ -99,14 +106,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStage);
-    uint64_t *full = bars;         // [2] stage loaded
-    uint64_t *empty = bars + 2;    // [2] stage consumed (P V done)
-    uint64_t *s_full = bars + 4;   // [2] S in TMEM
-    uint64_t *p_full = bars + 6;   // [2] P written (128 arrivals)
-    uint64_t *o_full = bars + 8;   // [2] O in TMEM
-    uint64_t *t_empty = bars + 10; // [2] O read out (128 arrivals)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint64_t *qk_full = bars;        // [2]
+    uint64_t *qk_empty = bars + 2;   // [2] S done
+    uint64_t *v_full = bars + 4;     // [3]
+    uint64_t *v_empty = bars + 7;    // [3] P V done
+    uint64_t *s_full = bars + 10;    // [2] S in TMEM buffer
+    uint64_t *p_full = bars + 12;    // [2] P in TMEM buffer (128 arrivals)
+    uint64_t *o_full = bars + 14;    // [2] O in TMEM buffer
+    uint64_t *t_empty = bars + 16;   // [2] TMEM buffer read out (128 arrivals)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -115,12 +124,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&full[i], 1);
-            tc::mbar_init(&empty[i], 1);
+            tc::mbar_init(&qk_full[i], 1);
+            tc::mbar_init(&qk_empty[i], 1);
             tc::mbar_init(&s_full[i], 1);
             tc::mbar_init(&p_full[i], kWG);
             tc::mbar_init(&o_full[i], 1);
             tc::mbar_init(&t_empty[i], kWG);
+        }
+        for (int i = 0; i < 3; ++i) {
+            tc::mbar_init(&v_full[i], 1);
+            tc::mbar_init(&v_empty[i], 1);
         }
         tc::fence_mbar_init();
         *abort_flag = 0;
@@ -135,41 +148,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wait_all = [&](uint64_t *bar, uint32_t parity) {
         return __all_sync(0xffffffffu, tc::mbar_wait_or_abort(bar, parity, p.err, abort_flag)) != 0;
     };
-    if (warp == kProducerWarp) {
+    if (warp == kQkWarp) {
         for (int i = 0; i < n_items; ++i) {
             const int s = i & 1;
-            if (i >= 2 && !wait_all(&empty[s], ((i >> 1) - 1) & 1)) break;
+            if (i >= 2 && !wait_all(&qk_empty[s], ((i >> 1) - 1) & 1)) break;
             if (lane == 0) {
                 const Item it = item_of(p, i);
-                uint8_t *st = smem + s * kStage;
-                tc::mbar_expect_tx(&full[s], kStage);
+                uint8_t *st = smem + s * kQkSlot;
+                tc::mbar_expect_tx(&qk_full[s], kQkSlot);
                 for (int half = 0; half < 2; ++half) {
-                    tc::tma_load_5d(st + half * kTile, &mq, &full[s], half * 64, it.head, it.w0, it.h0, it.t0);
-                    tc::tma_load_5d(st + (2 + half) * kTile, &mk, &full[s], half * 64, it.head, it.w0, it.h0, it.t0);
-                    tc::tma_load_5d(st + (4 + half) * kTile, &mv, &full[s], half * 64, it.head, it.w0, it.h0, it.t0);
+                    tc::tma_load_5d(st + half * kTile, &mq, &qk_full[s], half * 64, it.head, it.w0, it.h0, it.t0);
+                    tc::tma_load_5d(st + (2 + half) * kTile, &mk, &qk_full[s], half * 64, it.head, it.w0, it.h0, it.t0);
                 }
             }
             __syncwarp();
         }
+    } else if (warp == kVWarp) {
+        for (int i = 0; i < n_items; ++i) {
+            const int s = i % 3;
+            if (i >= 3 && !wait_all(&v_empty[s], ((i / 3) - 1) & 1)) break;
+            if (lane == 0) {
+                const Item it = item_of(p, i);
+                uint8_t *st = smem + kOffV + s * kVSlot;
+                tc::mbar_expect_tx(&v_full[s], kVSlot);
+                for (int half = 0; half < 2; ++half)
+                    tc::tma_load_5d(st + half * kTile, &mv, &v_full[s], half * 64, it.head, it.w0, it.h0, it.t0);
+            }
+            __syncwarp();
+        }
     } else if (warp == kMmaWarp) {
-        // S(i+1) is issued before waiting for P(i), so both warpgroups stay busy
         const uint32_t id_s = tc::idesc_bf16(128, 128, 0, 0);
         const uint32_t id_o = tc::idesc_bf16(128, 128, 0, 1);
         auto issue_s = [&](int i) -> bool {
-            const int s = i & 1;
+            const int b = i & 1;
             const uint32_t ph = (i >> 1) & 1;
-            if (!wait_all(&full[s], ph)) return false;
-            if (i >= 2 && !wait_all(&t_empty[s], ph ^ 1)) return false;
+            if (!wait_all(&qk_full[b], ph)) return false;
+            if (i >= 2 && !wait_all(&t_empty[b], ph ^ 1)) return false;
             tc::tc_fence_after();
             if (lane == 0) {
-                const uint32_t q0 = tc::smem_u32(smem + s * kStage), k0 = q0 + 2 * kTile;
+                const uint32_t q0 = tc::smem_u32(smem + b * kQkSlot), k0 = q0 + 2 * kTile;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t off = (k >> 2) * kTile + (k & 3) * 32;
-                    tc::mma_bf16(tmem + s * 256, tc::sdesc_sw128(q0 + off, 16, 1024), tc::sdesc_sw128(k0 + off, 16, 1024),
+                    tc::mma_bf16(tmem + b * 256, tc::sdesc_sw128(q0 + off, 16, 1024), tc::sdesc_sw128(k0 + off, 16, 1024),
                                  id_s, k > 0);
                 }
-                tc::mma_commit(&s_full[s]);
+                tc::mma_commit(&s_full[b]);
+                tc::mma_commit(&qk_empty[b]);
             }
             __syncwarp();
             return true;
@@ -177,25 +202,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n_items > 0 && issue_s(0)) {
             for (int i = 0; i < n_items; ++i) {
                 if (i + 1 < n_items && !issue_s(i + 1)) break;
-                const int s = i & 1;
-                if (!wait_all(&p_full[s], (i >> 1) & 1)) break;
+                const int b = i & 1, vs = i % 3;
+                if (!wait_all(&p_full[b], (i >> 1) & 1)) break;
+                if (!wait_all(&v_full[vs], (i / 3) & 1)) break;
                 tc::tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t p0 = tc::smem_u32(smem + s * kStage), v0 = p0 + 4 * kTile;
+                    const uint32_t v0 = tc::smem_u32(smem + kOffV + vs * kVSlot);
+                    const uint32_t tP = tmem + b * 256;  // P (bf16 pairs) over S
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t aoff = (k >> 2) * kTile + (k & 3) * 32;
-                        tc::mma_bf16(tmem + s * 256 + 128, tc::sdesc_sw128(p0 + aoff, 16, 1024),
-                                     tc::sdesc_sw128(v0 + k * 2048, kTile, 1024), id_o, k > 0);
-                    }
-                    tc::mma_commit(&o_full[s]);
-                    tc::mma_commit(&empty[s]);
+                    for (int k = 0; k < 8; ++k)
+                        tc::mma_bf16_tmem_a(tmem + b * 256 + 128, tP + k * 8, tc::sdesc_sw128(v0 + k * 2048, kTile, 1024),
+                                            id_o, k > 0);
+                    tc::mma_commit(&o_full[b]);
+                    tc::mma_commit(&v_empty[vs]);
                 }
                 __syncwarp();
             }
         }
-    } else {
-        // ---- warpgroup g handles the items i with i % 2 == g (stage and TMEM buffer g)
+    } else if (warp < 8) {
+        // ---- warpgroup g handles the items i with i % 2 == g (TMEM buffer g)
         const int g = warp >> 2, row = tid & (kWG - 1);
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
         const uint32_t tS = tmem + g * 256, tO = tS + 128;
@@ -219,33 +244,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < 32; ++j)
                     if ((kmask[c] >> j) & 1u) mx = fmaxf(mx, sv[j]);
             }
-            // pass 2: P = exp(S - max) as bf16 into the stage's Q tiles, and the row sum
+            // pass 2: P = exp(S - max) as bf16 pairs into TMEM columns 16c .. 16c+15,
+            // over S columns this thread has already read; and the row sum
             const float mxs = mx * p.scale_log2;
             float sum = 0.f;
-            uint8_t *pq = smem + g * kStage;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float sv[32];
                 tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv);
                 tc::tmem_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float e = ((kmask[c] >> j) & 1u) ? exp2f(fmaf(sv[j], p.scale_log2, -mxs)) : 0.f;
-                    sv[j] = e;
-                    sum += e;
+                for (int j = 0; j < 16; ++j) {
+                    const float e0 = ((kmask[c] >> (2 * j)) & 1u) ? exp2f(fmaf(sv[2 * j], p.scale_log2, -mxs)) : 0.f;
+                    const float e1 =
+                        ((kmask[c] >> (2 * j + 1)) & 1u) ? exp2f(fmaf(sv[2 * j + 1], p.scale_log2, -mxs)) : 0.f;
+                    sum += e0 + e1;
+                    pk[j] = tc::pack_bf16(e0, e1);
                 }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int key0 = c * 32 + q * 8;
-                    uint4 v;
-                    v.x = tc::pack_bf16(sv[q * 8 + 0], sv[q * 8 + 1]);
-                    v.y = tc::pack_bf16(sv[q * 8 + 2], sv[q * 8 + 3]);
-                    v.z = tc::pack_bf16(sv[q * 8 + 4], sv[q * 8 + 5]);
-                    v.w = tc::pack_bf16(sv[q * 8 + 6], sv[q * 8 + 7]);
-                    *reinterpret_cast<uint4 *>(pq + (key0 >> 6) * kTile + tc::sw128(row, (key0 & 63) >> 3)) = v;
-                }
+                tc::tmem_st16(tc::tmem_addr(tS, lane_base, c * 16), pk);
             }
-            tc::fence_proxy_async_smem();
+            tc::tmem_wait_st();
             tc::tc_fence_before();
             tc::mbar_arrive(&p_full[g]);
             const float inv = 1.f / sum;
