@@ -429,48 +429,52 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             const float ff = __expf(ci - rmid), fb = __expf(rmid - ei);
             const int wq = warp & 3;  // this warp's rows are 32*wq .. 32*wq + 31
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int j0 = 64 * g + 16 * qq;   // first of these 16 columns
-                uint32_t raw16[16];
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, j0), raw16);
+            for (int qp = 0; qp < 4; qp += 2) {
+                uint32_t raw2[2][16];  // two 16-column TMEM loads per wait
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp), raw2[0]);
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp + 16), raw2[1]);
                 tc::tmem_wait_ld();
-                float sv[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sv[e] = __uint_as_float(raw16[e]);
-                const int cc = j0 >> 5;             // 32-column block of these columns
-                if (factored && cc != wq) {         // off the diagonal block: one direction only
-                    // left of every row of this warp: forward; right of every row: flipped
-                    const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? sgf : sgb) + j0);
-                    const float rf = cc < wq ? ff : fb;
+                for (int u = 0; u < 2; ++u) {
+                    const int j0 = 64 * g + 16 * (qp + u);   // first of these 16 columns
+                    float sv[16];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 f4 = fac[q];
-                        sv[4 * q] *= rf * f4.x;
-                        sv[4 * q + 1] *= rf * f4.y;
-                        sv[4 * q + 2] *= rf * f4.z;
-                        sv[4 * q + 3] *= rf * f4.w;
+                    for (int e = 0; e < 16; ++e) sv[e] = __uint_as_float(raw2[u][e]);
+                    const int cc = j0 >> 5;             // 32-column block of these columns
+                    if (factored && cc != wq) {         // off the diagonal block: one direction only
+                        // left of every row of this warp: forward; right of every row: flipped
+                        const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? sgf : sgb) + j0);
+                        const float rf = cc < wq ? ff : fb;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 f4 = fac[q];
+                            sv[4 * q] *= rf * f4.x;
+                            sv[4 * q + 1] *= rf * f4.y;
+                            sv[4 * q + 2] *= rf * f4.z;
+                            sv[4 * q + 3] *= rf * f4.w;
+                        }
+                    } else if (factored) {              // the diagonal block
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int j = j0 + e;
+                            sv[e] *= (j <= r ? ff * sgf[j] : 0.f) + (j >= r ? fb * sgb[j] : 0.f);
+                        }
+                    } else {                            // decay range too wide: exact exponentials
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int j = j0 + e;
+                            const float cj = scum[k * kSub + j], dj = sdt[k * kSub + j];
+                            const float ej = cj - dj * Ah;
+                            sv[e] *= ((j <= r ? __expf(ci - cj) : 0.f) + (j >= r ? __expf(ej - ei) : 0.f)) * dj;
+                        }
                     }
-                } else if (factored) {              // the diagonal block
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int j = j0 + e;
-                        sv[e] *= (j <= r ? ff * sgf[j] : 0.f) + (j >= r ? fb * sgb[j] : 0.f);
-                    }
-                } else {                            // decay range too wide: exact exponentials
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int j = j0 + e;
-                        const float cj = scum[k * kSub + j], dj = sdt[k * kSub + j];
-                        const float ej = cj - dj * Ah;
-                        sv[e] *= ((j <= r ? __expf(ci - cj) : 0.f) + (j >= r ? __expf(ej - ei) : 0.f)) * dj;
-                    }
+                    uint8_t *tile = sM + g * kTile;
+                    const int ch = (j0 & 63) >> 3;
+                    *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch)) =
+                        make_uint4(bf2(sv[0], sv[1]), bf2(sv[2], sv[3]), bf2(sv[4], sv[5]), bf2(sv[6], sv[7]));
+                    *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch + 1)) =
+                        make_uint4(bf2(sv[8], sv[9]), bf2(sv[10], sv[11]), bf2(sv[12], sv[13]), bf2(sv[14], sv[15]));
                 }
-                uint8_t *tile = sM + g * kTile;
-                const int ch = (j0 & 63) >> 3;
-                *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch)) =
-                    make_uint4(bf2(sv[0], sv[1]), bf2(sv[2], sv[3]), bf2(sv[4], sv[5]), bf2(sv[6], sv[7]));
-                *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch + 1)) =
-                    make_uint4(bf2(sv[8], sv[9]), bf2(sv[10], sv[11]), bf2(sv[12], sv[13]), bf2(sv[14], sv[15]));
             }
         }
         {
@@ -519,11 +523,13 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             const bool valid = n < len;
             __nv_bfloat16 *dst =
                 static_cast<__nv_bfloat16 *>(a.out) + (((size_t)b * a.N + (valid ? sgoff[n] : 0)) * a.nh + h) * 64 + 32 * g;
+            uint32_t acc2[2][16];
+            tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g), acc2[0]);
+            tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g + 16), acc2[1]);
+            tc::tmem_wait_ld();
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
-                uint32_t acc[16];
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g + 16 * hq), acc);
-                tc::tmem_wait_ld();
+                const uint32_t *acc = acc2[hq];
                 if (valid) {
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {

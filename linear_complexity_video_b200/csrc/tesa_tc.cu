@@ -55,6 +55,7 @@ constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024 /*alignment slack*/;
 struct TesaTcParams {
     int T, H, W, nh;
     int Tw, Sw;
+    int sw_log2;        // log2(Sw) when Sw is a power of two, else -1
     int offt, offh, offw;
     int nwh, nww;
     int items;          // windows * heads
@@ -83,11 +84,27 @@ __device__ __forceinline__ Item item_of(const TesaTcParams &p, int local)
     return it;
 }
 
-// is box row r (r = (tt*Sw + hh)*Sw + ww) inside the grid?
+// grid coordinates of box row r (r = (tt*Sw + hh)*Sw + ww)
+__device__ __forceinline__ void row_coords(const TesaTcParams &p, const Item &it, int r, int &tt, int &hh, int &ww)
+{
+    if (p.sw_log2 >= 0) {
+        const int l = p.sw_log2;
+        tt = it.t0 + (r >> (2 * l));
+        hh = it.h0 + ((r >> l) & (p.Sw - 1));
+        ww = it.w0 + (r & (p.Sw - 1));
+    } else {
+        const int ss = p.Sw * p.Sw;
+        tt = it.t0 + r / ss;
+        hh = it.h0 + (r / p.Sw) % p.Sw;
+        ww = it.w0 + r % p.Sw;
+    }
+}
+
+// is box row r inside the grid?
 __device__ __forceinline__ bool row_in_grid(const TesaTcParams &p, const Item &it, int r)
 {
-    const int ss = p.Sw * p.Sw;
-    const int tt = it.t0 + r / ss, hh = it.h0 + (r / p.Sw) % p.Sw, ww = it.w0 + r % p.Sw;
+    int tt, hh, ww;
+    row_coords(p, it, r, tt, hh, ww);
     return tt >= 0 && tt < p.T && hh >= 0 && hh < p.H && ww >= 0 && ww < p.W;
 }
 
@@ -233,16 +250,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 4; ++c) kmask[c] = __ballot_sync(0xffffffffu, row_in_grid(p, it, c * 32 + lane));
             if (!wait_all(&s_full[g], ph)) break;
             tc::tc_fence_after();
-            // pass 1: row maximum over the keys in the grid
+            // pass 1: row maximum over the keys in the grid (two TMEM loads per wait)
             float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float sv[32];
-                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv);
+            for (int c = 0; c < 4; c += 2) {
+                float sv[2][32];
+                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv[0]);
+                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32 + 32), sv[1]);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if ((kmask[c] >> j) & 1u) mx = fmaxf(mx, sv[j]);
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if ((kmask[c + u] >> j) & 1u) mx = fmaxf(mx, sv[u][j]);
             }
             // pass 2: P = exp(S - max) as bf16 pairs into TMEM columns 16c .. 16c+15,
             // over S columns this thread has already read; and the row sum
@@ -272,26 +292,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             // epilogue: O row / sum -> global, once P V is done
             if (!wait_all(&o_full[g], ph)) break;
             tc::tc_fence_after();
-            const bool qvalid = row_in_grid(p, it, row);
-            const int ss = p.Sw * p.Sw;
-            const int tt = it.t0 + row / ss, hh = it.h0 + (row / p.Sw) % p.Sw, ww = it.w0 + row % p.Sw;
+            int tt, hh, ww;
+            row_coords(p, it, row, tt, hh, ww);
+            const bool qvalid = tt >= 0 && tt < p.T && hh >= 0 && hh < p.H && ww >= 0 && ww < p.W;
             __nv_bfloat16 *dst =
                 qvalid ? p.out + ((((size_t)tt * p.H + hh) * p.W + ww) * p.nh + it.head) * 128 : nullptr;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float o[32];
-                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, c * 32), o);
+            for (int c = 0; c < 4; c += 2) {
+                float o[2][32];
+                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, c * 32), o[0]);
+                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, c * 32 + 32), o[1]);
                 tc::tmem_wait_ld();
                 if (qvalid) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 v;
-                        v.x = tc::pack_bf16(o[q * 8 + 0] * inv, o[q * 8 + 1] * inv);
-                        v.y = tc::pack_bf16(o[q * 8 + 2] * inv, o[q * 8 + 3] * inv);
-                        v.z = tc::pack_bf16(o[q * 8 + 4] * inv, o[q * 8 + 5] * inv);
-                        v.w = tc::pack_bf16(o[q * 8 + 6] * inv, o[q * 8 + 7] * inv);
-                        *reinterpret_cast<uint4 *>(dst + c * 32 + q * 8) = v;
-                    }
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 v;
+                            v.x = tc::pack_bf16(o[u][q * 8 + 0] * inv, o[u][q * 8 + 1] * inv);
+                            v.y = tc::pack_bf16(o[u][q * 8 + 2] * inv, o[u][q * 8 + 3] * inv);
+                            v.z = tc::pack_bf16(o[u][q * 8 + 4] * inv, o[u][q * 8 + 5] * inv);
+                            v.w = tc::pack_bf16(o[u][q * 8 + 6] * inv, o[u][q * 8 + 7] * inv);
+                            *reinterpret_cast<uint4 *>(dst + (c + u) * 32 + q * 8) = v;
+                        }
                 }
             }
             tc::tc_fence_before();
@@ -370,6 +393,9 @@ cudaError_t launch_tesa_tc(const TesaArgs &a, cudaStream_t s)
     p.nh = a.nh;
     p.Tw = a.Tw;
     p.Sw = a.Sw;
+    p.sw_log2 = -1;
+    for (int l = 0; l < 8; ++l)
+        if ((1 << l) == a.Sw) p.sw_log2 = l;
     p.offt = a.offt;
     p.offh = a.offh;
     p.offw = a.offw;
