@@ -8,7 +8,7 @@
 //
 // One persistent CTA per SM walks (window, head) items. Q and K of an item sit
 // in one of two shared-memory slots that are released as soon as S = Q K^T is
-// done; V sits in one of three slots released after O = P V; P goes to TMEM
+// done; V sits in one of two slots released after O = P V; P goes to TMEM
 // over S (the A operand of P V is read from TMEM). Two warps issue the TMA
 // loads (Q+K and V), one warp issues tcgen05.mma, and two warpgroups take
 // turns with the softmax and the epilogue, so loads, tensor-core work and
@@ -22,8 +22,8 @@
 //   3. Thread i owns query i: it reads S row i from TMEM, masks keys outside
 //      the grid, and writes P = exp(S - max) as bf16 pairs back into TMEM.
 //   4. O = P V (P from TMEM, V as an MN-major shared-memory operand) into TMEM.
-//   5. Thread i scales O row i by 1 / sum(P) and stores it if query i is in
-//      the grid.
+//   5. Thread i scales O row i by 1 / sum(P); each warp stages its 32 rows in
+//      shared memory and stores those of queries in the grid as whole lines.
 // A window holds exactly one 128-token tile, so the softmax needs no online
 // rescaling.
 #include <cudaTypedefs.h>
@@ -40,11 +40,13 @@ namespace {
 
 constexpr uint32_t kTile = 16384;           // one 128-row x 128-byte box
 constexpr int kQkSlots = 2;                 // Q + K of an item (4 tiles), free once S = Q K^T is done
-constexpr int kVSlots = 3;                  // V of an item (2 tiles), free once O = P V is done
+constexpr int kVSlots = 2;                  // V of an item (2 tiles), free once O = P V is done
 constexpr uint32_t kQkSlot = 4 * kTile;
 constexpr uint32_t kVSlot = 2 * kTile;
 constexpr uint32_t kOffV = kQkSlots * kQkSlot;
-constexpr uint32_t kOffBar = kOffV + kVSlots * kVSlot;
+constexpr uint32_t kStage = 4096;          // per softmax warp: 32 rows x 128 B of O (bf16), swizzled
+constexpr uint32_t kOffStage = kOffV + kVSlots * kVSlot;
+constexpr uint32_t kOffBar = kOffStage + 8 * kStage;
 constexpr int kWG = 128;                    // a softmax / epilogue warpgroup
 constexpr int kQkWarp = 8;                  // TMA loads of Q and K
 constexpr int kVWarp = 9;                   // TMA loads of V
@@ -110,10 +112,11 @@ __device__ __forceinline__ bool row_in_grid(const TesaTcParams &p, const Item &i
 
 // Persistent CTA (one per SM) walking its share of the items.
 //   QK warp   : TMA Q and K of item i into QK slot i % 2 once S of item i-2 is done
-//   V warp    : TMA V of item i into V slot i % 3 once P V of item i-3 is done
-//   MMA warp  : S(i) = Q K^T into TMEM buffer i % 2 (once that buffer's previous
-//               item has been read out), then, one item behind, O = P V with P
-//               taken from TMEM (it overwrites S)
+//   V warp    : TMA V of item i into V slot i % 2 once P V of item i-2 is done
+//   MMA warp  : S(i) = Q K^T into the S columns of TMEM buffer i % 2 once P V of
+//               item i-2 has consumed the P held there; then, one item behind,
+//               O = P V with P taken from TMEM (P overwrites S), once the
+//               epilogue of item i-2 has read the O columns
 //   warpgroup g takes items i % 2 == g: softmax of S into P (bf16, in TMEM),
 //               then the epilogue O / rowsum -> global
 __global__ void __launch_bounds__(kThreads, 1)
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(&o_full[i], 1);
             tc::mbar_init(&t_empty[i], kWG);
         }
-        for (int i = 0; i < 3; ++i) {
+        for (int i = 0; i < kVSlots; ++i) {
             tc::mbar_init(&v_full[i], 1);
             tc::mbar_init(&v_empty[i], 1);
         }
@@ -182,8 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kVWarp) {
         for (int i = 0; i < n_items; ++i) {
-            const int s = i % 3;
-            if (i >= 3 && !wait_all(&v_empty[s], ((i / 3) - 1) & 1)) break;
+            const int s = i % kVSlots;
+            if (i >= kVSlots && !wait_all(&v_empty[s], ((i / kVSlots) - 1) & 1)) break;
             if (lane == 0) {
                 const Item it = item_of(p, i);
                 uint8_t *st = smem + kOffV + s * kVSlot;
@@ -200,7 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = i & 1;
             const uint32_t ph = (i >> 1) & 1;
             if (!wait_all(&qk_full[b], ph)) return false;
-            if (i >= 2 && !wait_all(&t_empty[b], ph ^ 1)) return false;
+            // S overwrites P of item i-2: wait until P V of that item is done
+            if (i >= 2 && !wait_all(&o_full[b], ph ^ 1)) return false;
             tc::tc_fence_after();
             if (lane == 0) {
                 const uint32_t q0 = tc::smem_u32(smem + b * kQkSlot), k0 = q0 + 2 * kTile;
@@ -219,9 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n_items > 0 && issue_s(0)) {
             for (int i = 0; i < n_items; ++i) {
                 if (i + 1 < n_items && !issue_s(i + 1)) break;
-                const int b = i & 1, vs = i % 3;
+                const int b = i & 1, vs = i % kVSlots;
                 if (!wait_all(&p_full[b], (i >> 1) & 1)) break;
-                if (!wait_all(&v_full[vs], (i / 3) & 1)) break;
+                if (!wait_all(&v_full[vs], (i / kVSlots) & 1)) break;
+                // O overwrites O of item i-2: wait until its epilogue has read it
+                if (i >= 2 && !wait_all(&t_empty[b], ((i >> 1) & 1) ^ 1)) break;
                 tc::tc_fence_after();
                 if (lane == 0) {
                     const uint32_t v0 = tc::smem_u32(smem + kOffV + vs * kVSlot);
@@ -248,38 +254,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t kmask[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) kmask[c] = __ballot_sync(0xffffffffu, row_in_grid(p, it, c * 32 + lane));
+            const bool all_keys = (kmask[0] & kmask[1] & kmask[2] & kmask[3]) == 0xffffffffu;
             if (!wait_all(&s_full[g], ph)) break;
             tc::tc_fence_after();
-            // pass 1: row maximum over the keys in the grid (two TMEM loads per wait)
-            float mx = -INFINITY;
+            // the whole S row in registers (one TMEM round trip)
+            float sv[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; c += 2) {
-                float sv[2][32];
-                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv[0]);
-                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32 + 32), sv[1]);
-                tc::tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv[c]);
+            tc::tmem_wait_ld();
+            if (!all_keys) {
+                // keys outside the grid (zero-filled rows) take no weight
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if ((kmask[c + u] >> j) & 1u) mx = fmaxf(mx, sv[u][j]);
+                        if (!((kmask[c] >> j) & 1u)) sv[c][j] = -INFINITY;
             }
-            // pass 2: P = exp(S - max) as bf16 pairs into TMEM columns 16c .. 16c+15,
-            // over S columns this thread has already read; and the row sum
+            // row maximum over eight independent chains
+            float m8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) m8[u] = fmaxf(sv[0][u], sv[0][u + 8]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (c > 0 || j >= 16) m8[j & 7] = fmaxf(m8[j & 7], sv[c][j]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            // P = 2^(S log2(e)/sqrt(d) - max') as bf16 pairs into TMEM columns
+            // 16c .. 16c+15 (over S columns already read), and the row sum
             const float mxs = mx * p.scale_log2;
-            float sum = 0.f;
+            float s8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s8[u] = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float sv[32];
-                tc::tmem_ld32(tc::tmem_addr(tS, lane_base, c * 32), sv);
-                tc::tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float e0 = ((kmask[c] >> (2 * j)) & 1u) ? exp2f(fmaf(sv[2 * j], p.scale_log2, -mxs)) : 0.f;
-                    const float e1 =
-                        ((kmask[c] >> (2 * j + 1)) & 1u) ? exp2f(fmaf(sv[2 * j + 1], p.scale_log2, -mxs)) : 0.f;
-                    sum += e0 + e1;
+                    const float e0 = tc::ex2_approx(fmaf(sv[c][2 * j], p.scale_log2, -mxs));
+                    const float e1 = tc::ex2_approx(fmaf(sv[c][2 * j + 1], p.scale_log2, -mxs));
+                    s8[(2 * j) & 7] += e0;
+                    s8[(2 * j + 1) & 7] += e1;
                     pk[j] = tc::pack_bf16(e0, e1);
                 }
                 tc::tmem_st16(tc::tmem_addr(tS, lane_base, c * 16), pk);
@@ -287,35 +303,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tmem_wait_st();
             tc::tc_fence_before();
             tc::mbar_arrive(&p_full[g]);
+            const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
             const float inv = 1.f / sum;
 
-            // epilogue: O row / sum -> global, once P V is done
+            // epilogue: O row / sum -> global, once P V is done. Each warp stages
+            // its 32 rows, 64 head dims at a time, in shared memory and writes
+            // them back as whole 128-byte lines (four rows per store instruction).
             if (!wait_all(&o_full[g], ph)) break;
             tc::tc_fence_after();
             int tt, hh, ww;
             row_coords(p, it, row, tt, hh, ww);
             const bool qvalid = tt >= 0 && tt < p.T && hh >= 0 && hh < p.H && ww >= 0 && ww < p.W;
-            __nv_bfloat16 *dst =
-                qvalid ? p.out + ((((size_t)tt * p.H + hh) * p.W + ww) * p.nh + it.head) * 128 : nullptr;
+            const size_t my_off = qvalid ? ((((size_t)tt * p.H + hh) * p.W + ww) * p.nh + it.head) * 128 : ~(size_t)0;
+            uint8_t *stage = smem + kOffStage + warp * kStage;
 #pragma unroll
-            for (int c = 0; c < 4; c += 2) {
+            for (int hf = 0; hf < 2; ++hf) {
                 float o[2][32];
-                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, c * 32), o[0]);
-                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, c * 32 + 32), o[1]);
+                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, hf * 64), o[0]);
+                tc::tmem_ld32(tc::tmem_addr(tO, lane_base, hf * 64 + 32), o[1]);
                 tc::tmem_wait_ld();
-                if (qvalid) {
 #pragma unroll
-                    for (int u = 0; u < 2; ++u)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 v;
-                            v.x = tc::pack_bf16(o[u][q * 8 + 0] * inv, o[u][q * 8 + 1] * inv);
-                            v.y = tc::pack_bf16(o[u][q * 8 + 2] * inv, o[u][q * 8 + 3] * inv);
-                            v.z = tc::pack_bf16(o[u][q * 8 + 4] * inv, o[u][q * 8 + 5] * inv);
-                            v.w = tc::pack_bf16(o[u][q * 8 + 6] * inv, o[u][q * 8 + 7] * inv);
-                            *reinterpret_cast<uint4 *>(dst + (c + u) * 32 + q * 8) = v;
-                        }
+                for (int q = 0; q < 8; ++q) {
+                    const int u = q >> 2, c0 = (q & 3) * 8;
+                    uint4 v;
+                    v.x = tc::pack_bf16(o[u][c0 + 0] * inv, o[u][c0 + 1] * inv);
+                    v.y = tc::pack_bf16(o[u][c0 + 2] * inv, o[u][c0 + 3] * inv);
+                    v.z = tc::pack_bf16(o[u][c0 + 4] * inv, o[u][c0 + 5] * inv);
+                    v.w = tc::pack_bf16(o[u][c0 + 6] * inv, o[u][c0 + 7] * inv);
+                    *reinterpret_cast<uint4 *>(stage + lane * 128 + ((q ^ (lane & 7)) << 4)) = v;
                 }
+                __syncwarp();
+                // lane l writes 16-byte piece (l % 8) of rows 4k + l / 8
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int rr = k * 4 + (lane >> 3), q = lane & 7;
+                    const size_t off = __shfl_sync(0xffffffffu, my_off, rr);
+                    const uint4 v = *reinterpret_cast<const uint4 *>(stage + rr * 128 + ((q ^ (rr & 7)) << 4));
+                    if (off != ~(size_t)0) *reinterpret_cast<uint4 *>(p.out + off + hf * 64 + q * 8) = v;
+                }
+                __syncwarp();
             }
             tc::tc_fence_before();
             tc::mbar_arrive(&t_empty[g]);
