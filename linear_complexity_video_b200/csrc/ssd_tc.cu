@@ -99,41 +99,6 @@ __device__ __forceinline__ void wait_loads(bool newer_pending)
         asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// 8 bf16 of a swizzled row -> floats
-__device__ __forceinline__ void row_chunk(const uint8_t *tile, int r, int c, float (&v)[8])
-{
-    const uint4 u = *reinterpret_cast<const uint4 *>(tile + tc::sw128(r, c));
-    float2 f;
-    f = tc::unpack_bf16(u.x); v[0] = f.x; v[1] = f.y;
-    f = tc::unpack_bf16(u.y); v[2] = f.x; v[3] = f.y;
-    f = tc::unpack_bf16(u.z); v[4] = f.x; v[5] = f.y;
-    f = tc::unpack_bf16(u.w); v[6] = f.x; v[7] = f.y;
-}
-
-__device__ __forceinline__ void put_chunk(uint8_t *tile, int r, int c, const float *v)
-{
-    uint4 u;
-    u.x = tc::pack_bf16(v[0], v[1]);
-    u.y = tc::pack_bf16(v[2], v[3]);
-    u.z = tc::pack_bf16(v[4], v[5]);
-    u.w = tc::pack_bf16(v[6], v[7]);
-    *reinterpret_cast<uint4 *>(tile + tc::sw128(r, c)) = u;
-}
-
-// max over the CTA (256 threads); `red` holds 8 floats
-__device__ __forceinline__ float block_max(float v, float *red)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float m = red[0];
-#pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
-    return m;
-}
-
 // Per-chunk setup shared by chunk_state and chunk_out: grid offsets and dt of
 // the chunk's L positions (zero past the sequence end).
 __device__ __forceinline__ void load_chunk_meta(const SsdArgs &a, int b, int h, int n0, int len, int L, int *goff,
@@ -243,6 +208,10 @@ __device__ __forceinline__ bool mma_wait(uint64_t *bar, uint32_t &phase, int *er
 //                           U_f / U_b (phase 1) or M (phase 3); h_f, h_b operands.
 //                           In phase 3, R_f C overwrites the C tile and R_b C the
 //                           B tile once S = C B^T is done.
+// Loads overlap math: phase 1 double-buffers x, B in the {x, B} and {C, h}
+// tiles; the chunk's entering states arrive during the last phase-1 sub-chunk;
+// the first output sub-chunk's rows load during phase 2 and each later one's
+// during the previous epilogue (x kept in registers for the 2 D x term).
 // ---------------------------------------------------------------------------
 constexpr uint32_t kOffX = 0;
 constexpr uint32_t kOffB = kTile;
@@ -253,8 +222,9 @@ constexpr uint32_t kOffDt = 6 * kTile;
 constexpr uint32_t kOffCum = kOffDt + kMaxChunk * 4;
 constexpr uint32_t kOffGoff = kOffCum + kMaxChunk * 4;
 constexpr uint32_t kOffGf = kOffGoff + kMaxChunk * 4;
-constexpr uint32_t kOffGb = kOffGf + kSub * 4;
-constexpr uint32_t kOffRed = kOffGb + kSub * 4;  // 8 floats
+constexpr uint32_t kOffGb = kOffGf + kMaxChunk * 4;
+constexpr uint32_t kOffRed = kOffGb + kMaxChunk * 4;  // 8 floats
+constexpr uint32_t kOffFlag = kOffRed + 32;           // kMaxSubs ints: sub-chunk takes the factored exps
 constexpr uint32_t kOffBar = kOffRed + 64;
 constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;
 
@@ -276,11 +246,12 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     float *sgf = reinterpret_cast<float *>(base + kOffGf);
     float *sgb = reinterpret_cast<float *>(base + kOffGb);
     float *sred = reinterpret_cast<float *>(base + kOffRed);
+    int *sflag = reinterpret_cast<int *>(base + kOffFlag);
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + kOffBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffBar + 8);
     int *abort_flag = reinterpret_cast<int *>(base + kOffBar + 12);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r = tid & (kSub - 1), g = tid >> 7;   // row / TMEM lane, column half
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
     const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
@@ -302,24 +273,59 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tR = tmem + kColR;
+    // x, B of sub-chunk 0 are in flight while the decay factors are prepared
+    load_rows(a, sX, sB, nullptr, sgoff, b, h, grp, len, 0);
     sub_cumsums(sdt, scum, Ah, nsub, false, sred);
+    // warp k: column factors of sub-chunk k around its midpoint r_k,
+    //   gf[n] = exp(r_k - c_n) dt_n, gb[n] = exp(e_n - r_k) dt_n,
+    // and whether every factor exponent of the sub-chunk stays within the limit
+    if (warp < nsub) {
+        const float rmid = scum[warp * kSub + kSub / 2 - 1];
+        float range = 0.f;
+#pragma unroll
+        for (int q = 0; q < kSub / 32; ++q) {
+            const int n = warp * kSub + q * 32 + lane;
+            const float cn = scum[n], dn = sdt[n], en = cn - dn * Ah;
+            sgf[n] = __expf(rmid - cn) * dn;
+            sgb[n] = __expf(en - rmid) * dn;
+            range = fmaxf(range, fmaxf(fabsf(cn - rmid), fabsf(en - rmid)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) range = fmaxf(range, __shfl_xor_sync(0xffffffffu, range, o));
+        if (lane == 0) sflag[warp] = range <= kFactorLimit;
+    }
 
     // ---------------- phase 1: sub-chunk-local states -> packed bf16 slots ------------
+    // x and B of sub-chunk k sit in buffer k % 2 ({x, B} tiles or {C, h} tiles);
+    // the next sub-chunk's rows load while this one is processed.
     for (int k = 0; k < nsub; ++k) {
-        load_rows(a, sX, sB, nullptr, sgoff, b, h, grp, len, k);
-        wait_loads(false);
+        uint8_t *tx = (k & 1) ? sC : sX, *tb = (k & 1) ? sHf : sB;
+        if (k + 1 < nsub) {
+            load_rows(a, (k & 1) ? sX : sC, (k & 1) ? sB : sHf, nullptr, sgoff, b, h, grp, len, k + 1);
+        } else {
+            // the chunk's entering states (fwd rows 0-63, flipped rows 64-127) into
+            // the free buffer's first tile: thread (r, g) copies its 64 bytes
+            const bool fwd = r < 64;
+            const char *Hin = reinterpret_cast<const char *>(fwd ? a.states_f : a.states_b) +
+                              (((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + (r & 63)) * 64 + 32 * g) * 2;
+            uint8_t *dst = ((k & 1) ? sX : sC) + r * 128 + g * 64;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tc::cp_async16(dst + 16 * q, Hin + 16 * q);
+            tc::cp_async_commit();
+        }
+        wait_loads(true);
         __syncthreads();
         {
             const int n = k * kSub + r;
             const float cj = scum[n], dj = sdt[n], cend = scum[k * kSub + kSub - 1];
-            build_u(sX, sM, sM + kTile, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
+            build_u(tx, sM, sM + kTile, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc::tc_fence_after();
-            mma_states(tR, tc::smem_u32(sM), tc::smem_u32(sB), false);
+            mma_states(tR, tc::smem_u32(sM), tc::smem_u32(tb), false);
             tc::mma_commit(bar);
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
@@ -342,21 +348,26 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     // ---------------- phase 2: chain the sub-chunk states ------------------------------
     {
         const bool fwd = r < 64;
-        const int p = fwd ? r : r - 64;
-        const __nv_bfloat16 *Hin = reinterpret_cast<const __nv_bfloat16 *>(fwd ? a.states_f : a.states_b) +
-                                   ((((size_t)b * a.nh + h) * a.nchunks + c) * 64 + p) * 64 + 32 * g;
         float hv[32];
+        wait_loads(false);
+        __syncthreads();
+        {
+            const uint8_t *src = ((nsub & 1) ? sC : sX) + r * 128 + g * 64;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(Hin + 8 * q);
-            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+            for (int q = 0; q < 4; ++q) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(src + 16 * q);
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = tc::unpack_bf16(w4[e]);
-                hv[8 * q + 2 * e] = f.x;
-                hv[8 * q + 2 * e + 1] = f.y;
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = tc::unpack_bf16(w4[e]);
+                    hv[8 * q + 2 * e] = f.x;
+                    hv[8 * q + 2 * e + 1] = f.y;
+                }
             }
         }
+        __syncthreads();
+        // x, B, C of the first output sub-chunk load during the chain
+        load_rows(a, sX, sB, sC, sgoff, b, h, grp, len, 0);
         for (int it = 0; it < nsub; ++it) {
             const int k = fwd ? it : nsub - 1 - it;
             const float alpha = __expf(scum[k * kSub + kSub - 1]);
@@ -382,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
 
     // ---------------- phase 3: outputs ---------------------------------------------
     for (int k = 0; k < nsub; ++k) {
-        load_rows(a, sX, sB, sC, sgoff, b, h, grp, len, k);
+        // (x, B, C of sub-chunk k were issued during the previous sub-chunk's epilogue)
         // entering states of sub-chunk k (already bf16) -> operand rows (forward if r < 64)
         {
             uint32_t pk[16];
@@ -400,12 +411,8 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
         const float ei = ci - di * Ah;
         const float cend = scum[k * kSub + kSub - 1];
         const float rmid = scum[k * kSub + kSub / 2 - 1];
-        if (g == 0) {
-            sgf[r] = __expf(rmid - ci) * di;  // forward column factor
-            sgb[r] = __expf(ei - rmid) * di;  // flipped column factor
-        }
-        const float range = block_max(g == 0 ? fmaxf(fabsf(ci - rmid), fabsf(ei - rmid)) : 0.f, sred);
-        const bool factored = range <= kFactorLimit;
+        const float *gf = sgf + k * kSub, *gb = sgb + k * kSub;  // column factors of this sub-chunk
+        const bool factored = sflag[k] != 0;
         wait_loads(false);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -443,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
                     const int cc = j0 >> 5;             // 32-column block of these columns
                     if (factored && cc != wq) {         // off the diagonal block: one direction only
                         // left of every row of this warp: forward; right of every row: flipped
-                        const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? sgf : sgb) + j0);
+                        const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? gf : gb) + j0);
                         const float rf = cc < wq ? ff : fb;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -457,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int j = j0 + e;
-                            sv[e] *= (j <= r ? ff * sgf[j] : 0.f) + (j >= r ? fb * sgb[j] : 0.f);
+                            sv[e] *= (j <= r ? ff * gf[j] : 0.f) + (j >= r ? fb * gb[j] : 0.f);
                         }
                     } else {                            // decay range too wide: exact exponentials
 #pragma unroll
@@ -517,31 +524,49 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
-        // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r -> grid position of token r.
-        // TMEM loads are warp-collective: every lane issues them, only real tokens store.
+        // this row's x (for the 2 D x term) to registers; then the next sub-chunk's
+        // x, B, C load into the tiles while the epilogue runs
+        uint4 xr[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xr[q] = *reinterpret_cast<const uint4 *>(sX + tc::sw128(r, 4 * g + q));
+        if (k + 1 < nsub) {
+            __syncthreads();
+            load_rows(a, sX, sB, sC, sgoff, b, h, grp, len, k + 1);
+        }
+
+        // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r, staged as bf16 in the
+        // (now free) M tile; then eight consecutive threads store each 128-byte row
+        // at the grid position of its token, so a warp writes four whole rows.
         {
-            const bool valid = n < len;
-            __nv_bfloat16 *dst =
-                static_cast<__nv_bfloat16 *>(a.out) + (((size_t)b * a.N + (valid ? sgoff[n] : 0)) * a.nh + h) * 64 + 32 * g;
             uint32_t acc2[2][16];
             tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g), acc2[0]);
             tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g + 16), acc2[1]);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {
-                const uint32_t *acc = acc2[hq];
-                if (valid) {
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t *acc = acc2[q >> 1] + 8 * (q & 1);
+                const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
+                uint32_t o4[4];
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        float xv[8];
-                        row_chunk(sX, r, 4 * g + 2 * hq + q, xv);
-                        uint32_t o4[4];
+                for (int e = 0; e < 4; ++e) {
+                    const float2 xv = tc::unpack_bf16(xw[e]);
+                    o4[e] = bf2(fmaf(Dh2, xv.x, __uint_as_float(acc[2 * e])),
+                                fmaf(Dh2, xv.y, __uint_as_float(acc[2 * e + 1])));
+                }
+                *reinterpret_cast<uint4 *>(sM + tc::sw128(r, 4 * g + q)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
+        }
+        __syncthreads();
+        {
+            const int ch = tid & 7;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o4[e] = bf2(fmaf(Dh2, xv[2 * e], __uint_as_float(acc[8 * q + 2 * e])),
-                                        fmaf(Dh2, xv[2 * e + 1], __uint_as_float(acc[8 * q + 2 * e + 1])));
-                        *reinterpret_cast<uint4 *>(dst + 16 * hq + 8 * q) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-                    }
+            for (int i = 0; i < kSub / (kThreads / 8); ++i) {
+                const int row = (tid >> 3) + i * (kThreads / 8), nn = k * kSub + row;
+                if (nn < len) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(sM + tc::sw128(row, ch));
+                    __nv_bfloat16 *dst =
+                        static_cast<__nv_bfloat16 *>(a.out) + (((size_t)b * a.N + sgoff[nn]) * a.nh + h) * 64 + ch * 8;
+                    *reinterpret_cast<uint4 *>(dst) = v;
                 }
             }
         }
