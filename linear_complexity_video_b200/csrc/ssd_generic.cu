@@ -79,60 +79,85 @@ __global__ void __launch_bounds__(kThreads) review_pool_kernel(SsdArgs a)
 
 // ---------------------------------------------------------------------------
 // review_pool, vectorised for bf16 storage: each thread sums one 16-byte vector
-// (8 channels of x or B) or one float4 of dt over the cell's box, with four
-// independent partial sums per channel for memory-level parallelism.
-// grid: (Np, ceil(vectors / 256), batch); needs nh*P % 8 == 0, G*Ns % 8 == 0,
-// nh % 4 == 0 and a 16-byte aligned dt.
+// (8 channels of x or B) or one float4 of dt over its part of the cell's box.
+// The block first lists the grid index of every token of that part in shared
+// memory (kPoolTokens at a time), so the summing loop has no index arithmetic
+// beyond one multiply-add per token, and it keeps eight 16-byte loads in
+// flight per thread.
+// grid: (Np, ceil(vectors / 256), batch * pool_splits); needs nh*P % 8 == 0,
+// G*Ns % 8 == 0, nh % 4 == 0 and a 16-byte aligned dt.
 // ---------------------------------------------------------------------------
+constexpr int kPoolTokens = 1024;
+constexpr int kPoolInFlight = 8;
+
 __global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
 {
+    __shared__ int s_tok[kPoolTokens];
     const int cell = blockIdx.x, b = blockIdx.z / a.pool_splits, sp = blockIdx.z % a.pool_splits;
     const int CX = a.nh * a.P, CD = a.nh, CB = a.G * a.Ns, CH = CX + CD + CB;
     const int VX = CX / 8, VB = CB / 8, VD = CD / 4;
     const int v = blockIdx.y * blockDim.x + threadIdx.x;
-    if (v >= VX + VB + VD) return;
+    const bool active = v < VX + VB + VD;
     const int hw = a.Hp * a.Wp;
     const int tp = cell / hw, r = cell - tp * hw, hp = r / a.Wp, wp = r - hp * a.Wp;
+    const int kind = v < VX ? 0 : (v < VX + VB ? 1 : 2);
+    // this thread's 16 bytes of token 0 of batch element b, and the token stride
+    const char *base;
+    size_t stride;
+    if (kind == 0) {
+        base = reinterpret_cast<const char *>(static_cast<const __nv_bfloat16 *>(a.x) + (size_t)b * a.N * CX + v * 8);
+        stride = (size_t)CX * 2;
+    } else if (kind == 1) {
+        base = reinterpret_cast<const char *>(static_cast<const __nv_bfloat16 *>(a.B) + (size_t)b * a.N * CB +
+                                              (v - VX) * 8);
+        stride = (size_t)CB * 2;
+    } else {
+        base = reinterpret_cast<const char *>(a.dt + (size_t)b * a.N * CD + (v - VX - VB) * 4);
+        stride = (size_t)CD * 4;
+    }
     int lo, hi;
     split_range(a.pt * a.ph * a.pw, a.pool_splits, sp, lo, hi);
-    const int kind = v < VX ? 0 : (v < VX + VB ? 1 : 2);
-    constexpr int kU = 4;  // tokens in flight per thread (8 costs occupancy: more registers)
-    float acc[kU][8];
+    float acc[8];
 #pragma unroll
-    for (int u = 0; u < kU; ++u)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
-    for (int i0 = lo; i0 < hi; i0 += kU) {
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int i = i0 + u;
-            if (i >= hi) break;
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int t0 = lo; t0 < hi; t0 += kPoolTokens) {
+        const int cnt = min(kPoolTokens, hi - t0);
+        __syncthreads();  // the previous list is no longer read
+        for (int q = threadIdx.x; q < cnt; q += blockDim.x) {
+            const int i = t0 + q;
             const int it = i / (a.ph * a.pw), rr = i - it * (a.ph * a.pw), ih = rr / a.pw, iw = rr - ih * a.pw;
-            const int g = ((tp * a.pt + it) * a.H + hp * a.ph + ih) * a.W + wp * a.pw + iw;
-            const size_t tok = (size_t)b * a.N + g;
-            if (kind == 2) {
-                const float4 d = *reinterpret_cast<const float4 *>(a.dt + tok * CD + (v - VX - VB) * 4);
-                acc[u][0] += d.x;
-                acc[u][1] += d.y;
-                acc[u][2] += d.z;
-                acc[u][3] += d.w;
-            } else {
-                const __nv_bfloat16 *src = kind == 0 ? static_cast<const __nv_bfloat16 *>(a.x) + tok * CX + v * 8
-                                                     : static_cast<const __nv_bfloat16 *>(a.B) + tok * CB + (v - VX) * 8;
-                const uint4 q = *reinterpret_cast<const uint4 *>(src);
-                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+            s_tok[q] = ((tp * a.pt + it) * a.H + hp * a.ph + ih) * a.W + wp * a.pw + iw;
+        }
+        __syncthreads();
+        if (!active) continue;
+        for (int q0 = 0; q0 < cnt; q0 += kPoolInFlight) {
+            uint4 w[kPoolInFlight];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[e]));
-                    acc[u][2 * e] += f.x;
-                    acc[u][2 * e + 1] += f.y;
+            for (int u = 0; u < kPoolInFlight; ++u)
+                w[u] = q0 + u < cnt ? *reinterpret_cast<const uint4 *>(base + (size_t)s_tok[q0 + u] * stride)
+                                    : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < kPoolInFlight; ++u) {
+                if (kind == 2) {
+                    acc[0] += __uint_as_float(w[u].x);
+                    acc[1] += __uint_as_float(w[u].y);
+                    acc[2] += __uint_as_float(w[u].z);
+                    acc[3] += __uint_as_float(w[u].w);
+                } else {
+                    // bf16 pair -> two floats: the low half shifted up, the high half masked
+                    acc[0] += __uint_as_float(w[u].x << 16);
+                    acc[1] += __uint_as_float(w[u].x & 0xffff0000u);
+                    acc[2] += __uint_as_float(w[u].y << 16);
+                    acc[3] += __uint_as_float(w[u].y & 0xffff0000u);
+                    acc[4] += __uint_as_float(w[u].z << 16);
+                    acc[5] += __uint_as_float(w[u].z & 0xffff0000u);
+                    acc[6] += __uint_as_float(w[u].w << 16);
+                    acc[7] += __uint_as_float(w[u].w & 0xffff0000u);
                 }
             }
         }
     }
-    float out[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
+    if (!active) return;
     float *dst = a.pooled + (((size_t)b * a.pool_splits + sp) * a.Np + cell) * CH;
     if (kind == 0) {
         dst += v * 8;
@@ -142,7 +167,9 @@ __global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
         dst += CX + (v - VX - VB) * 4;
     }
     const int n = kind == 2 ? 4 : 8;
-    for (int e = 0; e < n; ++e) dst[e] = out[e];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        if (e < n) dst[e] = acc[e];
 }
 
 // ---------------------------------------------------------------------------
