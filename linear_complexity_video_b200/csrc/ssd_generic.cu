@@ -175,7 +175,9 @@ __global__ void __launch_bounds__(kThreads) review_pool_vec_kernel(SsdArgs a)
 // ---------------------------------------------------------------------------
 // review_scan: h_init[b][h] = state after scanning [R, flip(R)] from zero,
 // R = pooled grid in scan order. The P rows of the state evolve independently,
-// so RS CTAs split them. grid: (nh, batch, RS)
+// so RS CTAs split them. The review tokens are staged RT positions at a time
+// (their grid cells listed first, so each value is one gather of the partial
+// box sums). grid: (nh, batch, RS)
 // ---------------------------------------------------------------------------
 template <int P, int NS, int RS>
 __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
@@ -183,9 +185,10 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
     constexpr int PR = P / RS;  // state rows of this CTA
     constexpr int PN = PR * NS;
     constexpr int E = (PN + kThreads - 1) / kThreads;
-    __shared__ float xs[kTile][PR];
-    __shared__ float bs[kTile][NS];
-    __shared__ float ds[kTile];
+    constexpr int W = PR + NS + 1;                            // x rows | B | dt per position
+    constexpr int RT = W * 128 * 4 <= 40 * 1024 ? 128 : 32;   // positions per staged tile
+    __shared__ float vals[RT][W];
+    __shared__ int cells[RT];
     const int h = blockIdx.x, b = blockIdx.y, p0 = blockIdx.z * PR;
     const int grp = h / (a.nh / a.G);
     const int CX = a.nh * a.P, CD = a.nh, CH = CX + CD + a.G * a.Ns;
@@ -195,37 +198,33 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
     float s[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) s[e] = 0.f;
-    for (int base = 0; base < L; base += kTile) {
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < kTile * (PR + NS + 1); idx += blockDim.x) {
-            const int k = idx / (PR + NS + 1), c = idx - k * (PR + NS + 1);
+    for (int base = 0; base < L; base += RT) {
+        __syncthreads();  // the previous tile is consumed
+        for (int k = threadIdx.x; k < RT; k += blockDim.x) {
             const int pos = base + k;
-            if (pos >= L) continue;
             const int r = pos < a.Np ? pos : L - 1 - pos;  // [R, flip(R)]
-            const int cell = rms_grid_offset(r, a.Tp, a.Hp, a.Wp, a.mode);
-            const int col = c < PR ? h * P + p0 + c : (c < PR + NS ? CX + CD + grp * NS + (c - PR) : CX + h);
-            float v = 0.f;
-            for (int sp = 0; sp < a.pool_splits; ++sp)
-                v += a.pooled[(((size_t)b * a.pool_splits + sp) * a.Np + cell) * CH + col];
-            v *= inv_box;
-            if (c < PR)
-                xs[k][c] = v;
-            else if (c < PR + NS)
-                bs[k][c - PR] = v;
-            else
-                ds[k] = v;
+            cells[k] = pos < L ? rms_grid_offset(r, a.Tp, a.Hp, a.Wp, a.mode) : 0;
         }
         __syncthreads();
-        const int kmax = min(kTile, L - base);
+        const int kmax = min(RT, L - base);
+        for (int idx = threadIdx.x; idx < kmax * W; idx += blockDim.x) {
+            const int k = idx / W, c = idx - k * W;
+            const int col = c < PR ? h * P + p0 + c : (c < PR + NS ? CX + CD + grp * NS + (c - PR) : CX + h);
+            const float *src = a.pooled + ((size_t)b * a.pool_splits * a.Np + cells[k]) * CH + col;
+            float v = 0.f;
+            for (int sp = 0; sp < a.pool_splits; ++sp) v += src[(size_t)sp * a.Np * CH];
+            vals[k][c] = v * inv_box;
+        }
+        __syncthreads();
         for (int k = 0; k < kmax; ++k) {
-            const float dk = ds[k];
+            const float dk = vals[k][PR + NS];
             const float dec = expf(dk * Ah);
 #pragma unroll
             for (int e = 0; e < E; ++e) {
                 const int idx = threadIdx.x + e * kThreads;
                 if (idx < PN) {
                     const int p = idx / NS, n = idx - p * NS;
-                    s[e] = dec * s[e] + dk * xs[k][p] * bs[k][n];
+                    s[e] = dec * s[e] + dk * vals[k][p] * vals[k][PR + n];
                 }
             }
         }
@@ -524,7 +523,7 @@ cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)
     }
     {
         Phase ph(MATE_PHASE_REVIEW_SCAN, s);
-        review_scan_kernel<64, 64, 4><<<dim3(a.nh, a.batch, 4), kThreads, 0, s>>>(a);
+        review_scan_kernel<64, 64, 8><<<dim3(a.nh, a.batch, 8), kThreads, 0, s>>>(a);
     }
     return cudaGetLastError();
 }

@@ -16,7 +16,7 @@
 //              with w_f[j] = exp(c_end - c_j) dt_j and w_b[j] = exp(e_j) dt_j
 //              (c, e: inclusive / exclusive cumulative sums of A dt over the
 //              chunk); rows 0-63 forward, rows 64-127 flipped.
-// state_chain  one thread per state element replaces every chunk-local state
+// state_chain  one thread per 8 state elements replaces every chunk-local state
 //              by the state entering the chunk (forward from the left, flipped
 //              from the right), starting from the review state or zero. The
 //              chunk states are stored as bf16 (halving their traffic); the
@@ -298,9 +298,12 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     // ---------------- phase 1: sub-chunk-local states -> packed bf16 slots ------------
     // x and B of sub-chunk k sit in buffer k % 2 ({x, B} tiles or {C, h} tiles);
     // the next sub-chunk's rows load while this one is processed.
+    wait_loads(false);
+    __syncthreads();
     for (int k = 0; k < nsub; ++k) {
         uint8_t *tx = (k & 1) ? sC : sX, *tb = (k & 1) ? sHf : sB;
         if (k + 1 < nsub) {
+            // buffer (k + 1) % 2 was last read by sub-chunk k - 1, whose MMA is done
             load_rows(a, (k & 1) ? sX : sC, (k & 1) ? sB : sHf, nullptr, sgoff, b, h, grp, len, k + 1);
         } else {
             // the chunk's entering states (fwd rows 0-63, flipped rows 64-127) into
@@ -313,8 +316,6 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             for (int q = 0; q < 4; ++q) tc::cp_async16(dst + 16 * q, Hin + 16 * q);
             tc::cp_async_commit();
         }
-        wait_loads(true);
-        __syncthreads();
         {
             const int n = k * kSub + r;
             const float cj = scum[n], dj = sdt[n], cend = scum[k * kSub + kSub - 1];
@@ -340,6 +341,8 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             tc::tmem_st16(tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g), pk);
             tc::tmem_wait_st();
         }
+        // the next sub-chunk's rows (or, after the last, the entering states) have landed
+        wait_loads(false);
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
@@ -349,8 +352,6 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     {
         const bool fwd = r < 64;
         float hv[32];
-        wait_loads(false);
-        __syncthreads();
         {
             const uint8_t *src = ((nsub & 1) ? sC : sX) + r * 128 + g * 64;
 #pragma unroll
@@ -387,25 +388,31 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             }
         }
     }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
 
     // ---------------- phase 3: outputs ---------------------------------------------
-    for (int k = 0; k < nsub; ++k) {
-        // (x, B, C of sub-chunk k were issued during the previous sub-chunk's epilogue)
-        // entering states of sub-chunk k (already bf16) -> operand rows (forward if r < 64)
-        {
-            uint32_t pk[16];
-            tc::tmem_ld16(tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g), pk);
-            tc::tmem_wait_ld();
-            uint8_t *ht = r < 64 ? sHf : sHb;
-            const int p = r & 63;
+    // Four barriers per sub-chunk: S done, M and R C written, Acc done (x rows read,
+    // so the next rows may load), and the epilogue done with the next rows landed.
+    //
+    // entering states of sub-chunk kk (already bf16) -> operand rows (forward if r < 64);
+    // each thread moves its own TMEM lane and columns
+    {
+    auto write_h = [&](int kk) {
+        uint32_t pk[16];
+        tc::tmem_ld16(tc::tmem_addr(tmem, lane_base, kk * 32 + 16 * g), pk);
+        tc::tmem_wait_ld();
+        uint8_t *ht = r < 64 ? sHf : sHb;
+        const int p = r & 63;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(ht + tc::sw128(p, 4 * g + q)) =
-                    make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(ht + tc::sw128(p, 4 * g + q)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    };
+    write_h(0);
+    wait_loads(false);
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    for (int k = 0; k < nsub; ++k) {
         const int n = k * kSub + r;
         const float ci = scum[n], di = sdt[n];
         const float ei = ci - di * Ah;
@@ -413,10 +420,6 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
         const float rmid = scum[k * kSub + kSub / 2 - 1];
         const float *gf = sgf + k * kSub, *gb = sgb + k * kSub;  // column factors of this sub-chunk
         const bool factored = sflag[k] != 0;
-        wait_loads(false);
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
 
         // S = C B^T -> TMEM R
         if (tid == 0) {
@@ -485,16 +488,16 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             }
         }
         {
-            // row r of C, scaled by R_f (g = 0, written over C) or R_b (g = 1, written over B)
-            const __nv_bfloat162 rs = __float2bfloat162_rn(g == 0 ? __expf(ci) : __expf(cend - ei));
-            uint4 cr[8];
+            // C row r, chunks 4g .. 4g+3 (this thread's own): R_f C over the C tile and
+            // R_b C over the B tile (free once S is done), in the same positions
+            const __nv_bfloat162 rf = __float2bfloat162_rn(__expf(ci)), rb = __float2bfloat162_rn(__expf(cend - ei));
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) cr[ch] = *reinterpret_cast<const uint4 *>(sC + tc::sw128(r, ch));
-            tc::tc_fence_before();
-            __syncthreads();  // every thread has its C row; S is consumed
-            uint8_t *dst = g == 0 ? sC : sB;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(dst + tc::sw128(r, ch)) = scale_chunk(cr[ch], rs);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t off = tc::sw128(r, 4 * g + q);
+                const uint4 cv = *reinterpret_cast<const uint4 *>(sC + off);
+                *reinterpret_cast<uint4 *>(sC + off) = scale_chunk(cv, rf);
+                *reinterpret_cast<uint4 *>(sB + off) = scale_chunk(cv, rb);
+            }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -522,26 +525,29 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
                              true);
             tc::mma_commit(bar);
         }
-        if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
-
-        // this row's x (for the 2 D x term) to registers; then the next sub-chunk's
-        // x, B, C load into the tiles while the epilogue runs
+        // this row's x (for the 2 D x term) to registers while the MMA runs (reads only)
         uint4 xr[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) xr[q] = *reinterpret_cast<const uint4 *>(sX + tc::sw128(r, 4 * g + q));
+        if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
+
+        // every tile is free: the next sub-chunk's states go to the h tiles and its
+        // x, B, C load while the epilogue runs
         if (k + 1 < nsub) {
-            __syncthreads();
+            write_h(k + 1);
             load_rows(a, sX, sB, sC, sgoff, b, h, grp, len, k + 1);
         }
 
-        // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r, staged as bf16 in the
-        // (now free) M tile; then eight consecutive threads store each 128-byte row
-        // at the grid position of its token, so a warp writes four whole rows.
+        // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r. Each warp stages its
+        // 32 half rows (64 bytes) in its own 2 KB of the free M tiles, then stores them
+        // at the grid positions of their tokens, eight half rows per store instruction.
         {
+            uint8_t *stg = sM + warp * 2048;
             uint32_t acc2[2][16];
             tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g), acc2[0]);
             tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g + 16), acc2[1]);
             tc::tmem_wait_ld();
+            const int lr = r & 31;  // this thread's row within the warp
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const uint32_t *acc = acc2[q >> 1] + 8 * (q & 1);
@@ -553,26 +559,28 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
                     o4[e] = bf2(fmaf(Dh2, xv.x, __uint_as_float(acc[2 * e])),
                                 fmaf(Dh2, xv.y, __uint_as_float(acc[2 * e + 1])));
                 }
-                *reinterpret_cast<uint4 *>(sM + tc::sw128(r, 4 * g + q)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                *reinterpret_cast<uint4 *>(stg + lr * 64 + ((q ^ ((lr >> 1) & 3)) << 4)) =
+                    make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
-        }
-        __syncthreads();
-        {
-            const int ch = tid & 7;
+            __syncwarp();
+            const int row0 = r & ~31;
 #pragma unroll
-            for (int i = 0; i < kSub / (kThreads / 8); ++i) {
-                const int row = (tid >> 3) + i * (kThreads / 8), nn = k * kSub + row;
+            for (int i = 0; i < 4; ++i) {
+                const int rr = i * 8 + (lane >> 2), q = lane & 3, nn = k * kSub + row0 + rr;
                 if (nn < len) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(sM + tc::sw128(row, ch));
-                    __nv_bfloat16 *dst =
-                        static_cast<__nv_bfloat16 *>(a.out) + (((size_t)b * a.N + sgoff[nn]) * a.nh + h) * 64 + ch * 8;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(stg + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4));
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
+                                         (((size_t)b * a.N + sgoff[nn]) * a.nh + h) * 64 + 32 * g + q * 8;
                     *reinterpret_cast<uint4 *>(dst) = v;
                 }
             }
         }
+        if (k + 1 < nsub) wait_loads(false);
+        tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
+    }
     }
 
 cleanup:
@@ -687,46 +695,60 @@ done:
 }
 
 // ---------------------------------------------------------------------------
-// state_chain: one thread per element of the 64 x 64 state. The chunk states
-// are stored as bf16; the chain itself runs in fp32.
-// grid: (4096 / 256, nh * batch, 2 directions)
+// state_chain: one thread per eight consecutive elements of the 64 x 64 state
+// (one 16-byte vector). The chunk states are stored as bf16; the chain itself
+// runs in fp32, with the loads of kAhead chunks in flight ahead of it.
+// grid: (4096 / 8 / 256, nh * batch, 2 directions)
 // ---------------------------------------------------------------------------
 constexpr int kAhead = 8;
 
 __global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
 {
-    const int e = blockIdx.x * 256 + threadIdx.x;
+    const int e8 = (blockIdx.x * 256 + threadIdx.x) * 8;  // first of this thread's 8 elements
     const int hb = blockIdx.y, dir = blockIdx.z;
     const int h = hb % a.nh, b = hb / a.nh;
     const int nc = a.nchunks;
     __nv_bfloat16 *S = reinterpret_cast<__nv_bfloat16 *>(dir == 0 ? a.states_f : a.states_b) +
-                       ((size_t)b * a.nh + h) * nc * 4096 + e;
+                       ((size_t)b * a.nh + h) * nc * 4096 + e8;
     const float *al = a.alpha + ((size_t)b * a.nh + h) * nc;
-    float hv = a.review ? a.h_init[((size_t)b * a.nh + h) * 4096 + e] : 0.f;
+    float hv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hv[j] = a.review ? a.h_init[((size_t)b * a.nh + h) * 4096 + e8 + j] : 0.f;
+    // one chain step: the stored chunk-local state becomes the entering state
+    auto step_chunk = [&](int cidx, uint4 loc, float alpha) {
+        uint4 o;
+        o.x = tc::pack_bf16(hv[0], hv[1]);
+        o.y = tc::pack_bf16(hv[2], hv[3]);
+        o.z = tc::pack_bf16(hv[4], hv[5]);
+        o.w = tc::pack_bf16(hv[6], hv[7]);
+        *reinterpret_cast<uint4 *>(S + (size_t)cidx * 4096) = o;
+        const uint32_t w4[4] = {loc.x, loc.y, loc.z, loc.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = tc::unpack_bf16(w4[q]);
+            hv[2 * q] = fmaf(alpha, hv[2 * q], f.x);
+            hv[2 * q + 1] = fmaf(alpha, hv[2 * q + 1], f.y);
+        }
+    };
     // visit chunks in chain order: forward 0 .. nc-1, flipped nc-1 .. 0
     const int step = dir == 0 ? 1 : -1;
     int cidx = dir == 0 ? 0 : nc - 1;
     int left = nc;
     while (left >= kAhead) {
-        float buf[kAhead], alp[kAhead];
+        uint4 buf[kAhead];
+        float alp[kAhead];
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) {
-            buf[u] = __bfloat162float(S[(size_t)(cidx + u * step) * 4096]);
+            buf[u] = *reinterpret_cast<const uint4 *>(S + (size_t)(cidx + u * step) * 4096);
             alp[u] = al[cidx + u * step];
         }
 #pragma unroll
-        for (int u = 0; u < kAhead; ++u) {
-            S[(size_t)(cidx + u * step) * 4096] = __float2bfloat16_rn(hv);
-            hv = fmaf(alp[u], hv, buf[u]);
-        }
+        for (int u = 0; u < kAhead; ++u) step_chunk(cidx + u * step, buf[u], alp[u]);
         cidx += kAhead * step;
         left -= kAhead;
     }
-    for (; left > 0; --left, cidx += step) {
-        const float v = __bfloat162float(S[(size_t)cidx * 4096]);
-        S[(size_t)cidx * 4096] = __float2bfloat16_rn(hv);
-        hv = fmaf(al[cidx], hv, v);
-    }
+    for (; left > 0; --left, cidx += step)
+        step_chunk(cidx, *reinterpret_cast<const uint4 *>(S + (size_t)cidx * 4096), al[cidx]);
 }
 
 }  // namespace
@@ -757,7 +779,7 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
     }
     {
         Phase ph(MATE_PHASE_STATE_PASS, s);
-        ssd_state_chain_kernel<<<dim3(4096 / 256, a.nh * a.batch, 2), 256, 0, s>>>(a);
+        ssd_state_chain_kernel<<<dim3(4096 / 8 / 256, a.nh * a.batch, 2), 256, 0, s>>>(a);
     }
     {
         Phase ph(MATE_PHASE_CHUNK_OUT, s);
