@@ -207,31 +207,57 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
         }
         __syncthreads();
         const int kmax = min(RT, L - base);
-        for (int idx = threadIdx.x; idx < kmax * W; idx += blockDim.x) {
-            const int k = idx / W, c = idx - k * W;
-            const int col = c < PR ? h * P + p0 + c : (c < PR + NS ? CX + CD + grp * NS + (c - PR) : CX + h);
-            const float *src = a.pooled + ((size_t)b * a.pool_splits * a.Np + cells[k]) * CH + col;
-            float v = 0.f;
-            for (int sp = 0; sp < a.pool_splits; ++sp) v += src[(size_t)sp * a.Np * CH];
-            vals[k][c] = v * inv_box;
+        // eight gathers in flight per thread
+        constexpr int kU = 8;
+        for (int i0 = threadIdx.x; i0 < kmax * W; i0 += kU * blockDim.x) {
+            const float *src[kU];
+            float v[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int idx = min(i0 + u * (int)blockDim.x, kmax * W - 1);
+                const int k = idx / W, c = idx - k * W;
+                const int col = c < PR ? h * P + p0 + c : (c < PR + NS ? CX + CD + grp * NS + (c - PR) : CX + h);
+                src[u] = a.pooled + ((size_t)b * a.pool_splits * a.Np + cells[k]) * CH + col;
+                v[u] = 0.f;
+            }
+            for (int sp = 0; sp < a.pool_splits; ++sp)
+#pragma unroll
+                for (int u = 0; u < kU; ++u) v[u] += src[u][(size_t)sp * a.Np * CH];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int idx = i0 + u * (int)blockDim.x;
+                if (idx < kmax * W) {
+                    const int k = idx / W, c = idx - k * W;
+                    vals[k][c] = v[u] * inv_box;
+                }
+            }
         }
         __syncthreads();
-        for (int k = 0; k < kmax; ++k) {
+        // per position: the decay exp(dt A) (kept in the dt slot) and dt x
+        for (int k = threadIdx.x; k < kmax; k += blockDim.x) {
             const float dk = vals[k][PR + NS];
-            const float dec = expf(dk * Ah);
+#pragma unroll
+            for (int p = 0; p < PR; ++p) vals[k][p] *= dk;
+            vals[k][PR + NS] = expf(dk * Ah);
+        }
+        __syncthreads();
+        // thread t owns the E consecutive elements t*E .. of the PR x NS block
+        // (one state row p, adjacent columns n)
+        for (int k = 0; k < kmax; ++k) {
+            const float dec = vals[k][PR + NS];
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const int idx = threadIdx.x + e * kThreads;
+                const int idx = threadIdx.x * E + e;
                 if (idx < PN) {
                     const int p = idx / NS, n = idx - p * NS;
-                    s[e] = dec * s[e] + dk * vals[k][p] * vals[k][PR + n];
+                    s[e] = fmaf(dec, s[e], vals[k][p] * vals[k][PR + n]);
                 }
             }
         }
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-        const int idx = threadIdx.x + e * kThreads;
+        const int idx = threadIdx.x * E + e;
         if (idx < PN) a.h_init[((size_t)b * a.nh + h) * (P * NS) + p0 * NS + idx] = s[e];
     }
 }
