@@ -41,6 +41,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
+#include "tmap.h"
 
 namespace mate {
 
@@ -89,6 +90,28 @@ __device__ __forceinline__ void load_rows(const SsdArgs &a, uint8_t *tX, uint8_t
         }
     }
     tc::cp_async_commit();
+}
+
+// Where the scan order makes every 128-position sub-chunk a box of the grid,
+// its x, B, C rows come by TMA (one box each, already in the 128-byte swizzle)
+// instead of per-thread gathers. One kernel launch per batch element then.
+struct TmaRows {
+    int use;      // 1: TMA boxes
+    int n0, n1;   // scan axis lengths, fastest first
+    int zbase;    // batch element of blockIdx.z == 0
+};
+
+// issued by one thread: x (channel h) and B, C (channel grp; tC may be null) rows
+// of the sub-chunk starting at scan position s, completing on `bar`
+__device__ __forceinline__ void tma_rows(const CUtensorMap *mx, const CUtensorMap *mb, const CUtensorMap *mc,
+                                         const TmaRows &g, uint8_t *tX, uint8_t *tB, uint8_t *tC, uint64_t *bar,
+                                         int h, int grp, int s)
+{
+    const int a0 = s % g.n0, q = s / g.n0, a1 = q % g.n1, a2 = q / g.n1;
+    tc::mbar_expect_tx(bar, (tC ? 3u : 2u) * kTile);
+    tc::tma_load_5d(tX, mx, bar, 0, h, a0, a1, a2);
+    tc::tma_load_5d(tB, mb, bar, 0, grp, a0, a1, a2);
+    if (tC) tc::tma_load_5d(tC, mc, bar, 0, grp, a0, a1, a2);
 }
 
 __device__ __forceinline__ void wait_loads(bool newer_pending)
@@ -233,7 +256,9 @@ constexpr uint32_t kTmemCols = 256;
 
 __device__ __forceinline__ uint32_t bf2(float lo, float hi) { return tc::pack_bf16(lo, hi); }
 
-__global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a, int nsub)
+__global__ void __launch_bounds__(kThreads, 2)
+    ssd_chunk_out_tc_kernel(SsdArgs a, int nsub, const __grid_constant__ CUtensorMap mx,
+                            const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC, TmaRows geo)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
@@ -250,20 +275,22 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + kOffBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffBar + 8);
     int *abort_flag = reinterpret_cast<int *>(base + kOffBar + 12);
+    uint64_t *ldbar = reinterpret_cast<uint64_t *>(base + kOffBar + 16);  // TMA row loads
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r = tid & (kSub - 1), g = tid >> 7;   // row / TMEM lane, column half
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z + geo.zbase;
     const int L = nsub * kSub;
     const int n0 = c * L, len = min(L, a.N - n0);
     const int grp = h / (a.nh / a.G);
     const float Ah = a.A[h], Dh2 = 2.f * a.D[h];
-    uint32_t mma_phase = 0;
+    uint32_t mma_phase = 0, ld_issued = 0, ld_phase = 0;  // TMA batches issued / completed
 
     if (warp == 0) tc::tmem_alloc(tmem_slot, kTmemCols);
     if (tid == 0) {
         tc::mbar_init(bar, 1);
+        tc::mbar_init(ldbar, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
@@ -273,8 +300,31 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tR = tmem + kColR;
+    // rows of sub-chunk `sub` into the given tiles: a TMA batch from one thread, or
+    // per-thread cp.async gathers
+    auto issue_rows = [&](uint8_t *tx, uint8_t *tb, uint8_t *tcc, int sub) {
+        if (geo.use) {
+            if (tid == 0) tma_rows(&mx, &mB, &mC, geo, tx, tb, tcc, ldbar, h, grp, n0 + sub * kSub);
+            ++ld_issued;
+        } else {
+            load_rows(a, tx, tb, tcc, sgoff, b, h, grp, len, sub);
+        }
+    };
+    // waits for the pending TMA batch (at most one) and every cp.async group, then a
+    // CTA barrier; false (on every thread) once a wait has timed out
+    auto rows_wait = [&]() {
+        if (ld_issued > ld_phase) {
+            if (tc::mbar_wait(ldbar, ld_phase & 1u, a.err))
+                ++ld_phase;
+            else
+                *abort_flag = 1;
+        }
+        tc::cp_async_wait_all();
+        __syncthreads();
+        return *abort_flag == 0;
+    };
     // x, B of sub-chunk 0 are in flight while the decay factors are prepared
-    load_rows(a, sX, sB, nullptr, sgoff, b, h, grp, len, 0);
+    issue_rows(sX, sB, nullptr, 0);
     sub_cumsums(sdt, scum, Ah, nsub, false, sred);
     // warp k: column factors of sub-chunk k around its midpoint r_k,
     //   gf[n] = exp(r_k - c_n) dt_n, gb[n] = exp(e_n - r_k) dt_n,
@@ -298,13 +348,12 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
     // ---------------- phase 1: sub-chunk-local states -> packed bf16 slots ------------
     // x and B of sub-chunk k sit in buffer k % 2 ({x, B} tiles or {C, h} tiles);
     // the next sub-chunk's rows load while this one is processed.
-    wait_loads(false);
-    __syncthreads();
+    if (!rows_wait()) goto cleanup;
     for (int k = 0; k < nsub; ++k) {
         uint8_t *tx = (k & 1) ? sC : sX, *tb = (k & 1) ? sHf : sB;
         if (k + 1 < nsub) {
             // buffer (k + 1) % 2 was last read by sub-chunk k - 1, whose MMA is done
-            load_rows(a, (k & 1) ? sX : sC, (k & 1) ? sB : sHf, nullptr, sgoff, b, h, grp, len, k + 1);
+            issue_rows((k & 1) ? sX : sC, (k & 1) ? sB : sHf, nullptr, k + 1);
         } else {
             // the chunk's entering states (fwd rows 0-63, flipped rows 64-127) into
             // the free buffer's first tile: thread (r, g) copies its 64 bytes
@@ -342,9 +391,8 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
             tc::tmem_wait_st();
         }
         // the next sub-chunk's rows (or, after the last, the entering states) have landed
-        wait_loads(false);
         tc::tc_fence_before();
-        __syncthreads();
+        if (!rows_wait()) goto cleanup;
         tc::tc_fence_after();
     }
 
@@ -366,26 +414,34 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
                 }
             }
         }
+        tc::fence_proxy_async_smem();
         __syncthreads();
         // x, B, C of the first output sub-chunk load during the chain
-        load_rows(a, sX, sB, sC, sgoff, b, h, grp, len, 0);
-        for (int it = 0; it < nsub; ++it) {
-            const int k = fwd ? it : nsub - 1 - it;
-            const float alpha = __expf(scum[k * kSub + kSub - 1]);
-            const uint32_t ta = tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g);
-            uint32_t loc[16], pk[16];
-            tc::tmem_ld16(ta, loc);
+        issue_rows(sX, sB, sC, 0);
+        // two slots per TMEM round trip (loads of both, then stores of both)
+        for (int it0 = 0; it0 < nsub; it0 += 2) {
+            const bool two = it0 + 1 < nsub;
+            const int k0 = fwd ? it0 : nsub - 1 - it0, k1 = fwd ? it0 + 1 : nsub - 2 - it0;
+            uint32_t loc[2][16], pk[2][16];  // separate sources for the two stores in flight
+            tc::tmem_ld16(tc::tmem_addr(tmem, lane_base, k0 * 32 + 16 * g), loc[0]);
+            if (two) tc::tmem_ld16(tc::tmem_addr(tmem, lane_base, k1 * 32 + 16 * g), loc[1]);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) pk[q] = bf2(hv[2 * q], hv[2 * q + 1]);
-            tc::tmem_st16(ta, pk);
-            tc::tmem_wait_st();
+            for (int u = 0; u < 2; ++u) {
+                if (u == 1 && !two) break;
+                const int k = u == 0 ? k0 : k1;
+                const float alpha = __expf(scum[k * kSub + kSub - 1]);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float2 f = tc::unpack_bf16(loc[q]);
-                hv[2 * q] = fmaf(alpha, hv[2 * q], f.x);
-                hv[2 * q + 1] = fmaf(alpha, hv[2 * q + 1], f.y);
+                for (int q = 0; q < 16; ++q) pk[u][q] = bf2(hv[2 * q], hv[2 * q + 1]);
+                tc::tmem_st16(tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g), pk[u]);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float2 f = tc::unpack_bf16(loc[u][q]);
+                    hv[2 * q] = fmaf(alpha, hv[2 * q], f.x);
+                    hv[2 * q + 1] = fmaf(alpha, hv[2 * q + 1], f.y);
+                }
             }
+            tc::tmem_wait_st();
         }
     }
 
@@ -408,10 +464,9 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
     };
     write_h(0);
-    wait_loads(false);
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
-    __syncthreads();
+    if (!rows_wait()) goto cleanup;
     for (int k = 0; k < nsub; ++k) {
         const int n = k * kSub + r;
         const float ci = scum[n], di = sdt[n];
@@ -529,13 +584,14 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
         uint4 xr[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) xr[q] = *reinterpret_cast<const uint4 *>(sX + tc::sw128(r, 4 * g + q));
+        tc::fence_proxy_async_smem();  // those reads precede the next rows' TMA writes
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
         // every tile is free: the next sub-chunk's states go to the h tiles and its
         // x, B, C load while the epilogue runs
         if (k + 1 < nsub) {
             write_h(k + 1);
-            load_rows(a, sX, sB, sC, sgoff, b, h, grp, len, k + 1);
+            issue_rows(sX, sB, sC, k + 1);
         }
 
         // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r. Each warp stages its
@@ -575,16 +631,17 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_chunk_out_tc_kernel(SsdArgs a
                 }
             }
         }
-        if (k + 1 < nsub) wait_loads(false);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        __syncthreads();
+        if (!rows_wait()) goto cleanup;
         tc::tc_fence_after();
     }
     }
 
 cleanup:
     tc::cp_async_wait_all();
+    // after a timeout a TMA batch may still be landing: a second bounded wait for it
+    if (ld_issued > ld_phase && tid == 0) tc::mbar_wait(ldbar, ld_phase & 1u, nullptr);
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -608,7 +665,9 @@ constexpr uint32_t kStOffRed = kStOffGoff + kMaxChunk * 4;  // 8 floats
 constexpr uint32_t kStOffBar = kStOffRed + 64;
 constexpr uint32_t kStSmemBytes = kStOffBar + 64 + 1024;
 
-__global__ void __launch_bounds__(kThreads, 4) ssd_chunk_state_tc_kernel(SsdArgs a, int nsub)
+__global__ void __launch_bounds__(kThreads, 4)
+    ssd_chunk_state_tc_kernel(SsdArgs a, int nsub, const __grid_constant__ CUtensorMap mx,
+                              const __grid_constant__ CUtensorMap mB, TmaRows geo)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
@@ -621,20 +680,22 @@ __global__ void __launch_bounds__(kThreads, 4) ssd_chunk_state_tc_kernel(SsdArgs
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + kStOffBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kStOffBar + 8);
     int *abort_flag = reinterpret_cast<int *>(base + kStOffBar + 12);
+    uint64_t *ldbar = reinterpret_cast<uint64_t *>(base + kStOffBar + 16);  // TMA row loads
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int r = tid & (kSub - 1), g = tid >> 7;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z + geo.zbase;
     const int L = nsub * kSub;
     const int n0 = c * L, len = min(L, a.N - n0);
     const int grp = h / (a.nh / a.G);
     const float Ah = a.A[h];
-    uint32_t mma_phase = 0;
+    uint32_t mma_phase = 0, ld_issued = 0, ld_phase = 0;  // TMA batches issued / completed
 
     if (warp == 0) tc::tmem_alloc(tmem_slot, 64);
     if (tid == 0) {
         tc::mbar_init(bar, 1);
+        tc::mbar_init(ldbar, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
@@ -647,9 +708,19 @@ __global__ void __launch_bounds__(kThreads, 4) ssd_chunk_state_tc_kernel(SsdArgs
     const float cend = scum[L - 1];
 
     for (int k = 0; k < nsub; ++k) {
-        load_rows(a, tX, tB, nullptr, sgoff, b, h, grp, len, k);
-        wait_loads(false);
+        if (geo.use) {
+            if (tid == 0) tma_rows(&mx, &mB, nullptr, geo, tX, tB, nullptr, ldbar, h, grp, n0 + k * kSub);
+            ++ld_issued;
+            if (tc::mbar_wait(ldbar, ld_phase & 1u, a.err))
+                ++ld_phase;
+            else
+                *abort_flag = 1;
+        } else {
+            load_rows(a, tX, tB, nullptr, sgoff, b, h, grp, len, k);
+            wait_loads(false);
+        }
         __syncthreads();
+        if (*abort_flag) goto done;
         {
             const int n = k * kSub + r;
             const float cj = scum[n], dj = sdt[n];
@@ -686,6 +757,8 @@ __global__ void __launch_bounds__(kThreads, 4) ssd_chunk_state_tc_kernel(SsdArgs
     }
 done:
     tc::cp_async_wait_all();
+    // after a timeout a TMA batch may still be landing: a second bounded wait for it
+    if (ld_issued > ld_phase && tid == 0) tc::mbar_wait(ldbar, ld_phase & 1u, nullptr);
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -773,17 +846,52 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
         if (e != cudaSuccess) return e;
     }
     const int nsub = a.Q / kSub;
-    {
+    // TMA row boxes when the scan order allows them: one launch per batch element
+    struct Maps {
+        CUtensorMap x, b, c;
+    };
+    const ScanBox sb = scan_box(a.mode, a.T, a.H, a.W);
+    auto build_maps = [&](int bb, Maps &m) {
+        const uint64_t tx = (uint64_t)a.nh * 64 * 2, tb = (uint64_t)a.G * 64 * 2;  // token strides in bytes
+        const uint64_t dx[5] = {64, (uint64_t)a.nh, (uint64_t)sb.n[0], (uint64_t)sb.n[1], (uint64_t)sb.n[2]};
+        const uint64_t db[5] = {64, (uint64_t)a.G, (uint64_t)sb.n[0], (uint64_t)sb.n[1], (uint64_t)sb.n[2]};
+        const uint64_t sx[4] = {128, sb.stride[0] * tx, sb.stride[1] * tx, sb.stride[2] * tx};
+        const uint64_t sbs[4] = {128, sb.stride[0] * tb, sb.stride[1] * tb, sb.stride[2] * tb};
+        const uint32_t box[5] = {64, 1, sb.box[0], sb.box[1], sb.box[2]};
+        const size_t tok = (size_t)bb * a.N;
+        return tmap_bf16_5d(&m.x, static_cast<const __nv_bfloat16 *>(a.x) + tok * a.nh * 64, dx, sx, box) &&
+               tmap_bf16_5d(&m.b, static_cast<const __nv_bfloat16 *>(a.B) + tok * a.G * 64, db, sbs, box) &&
+               tmap_bf16_5d(&m.c, static_cast<const __nv_bfloat16 *>(a.C) + tok * a.G * 64, db, sbs, box);
+    };
+    Maps maps = {};
+    TmaRows geo = {0, 1, 1, 0};
+    if (sb.ok && tmap_available() && build_maps(0, maps)) {
+        geo.use = 1;
+        geo.n0 = sb.n[0];
+        geo.n1 = sb.n[1];
+    }
+    const int launches = geo.use ? a.batch : 1, zdim = geo.use ? 1 : a.batch;
+    for (int l = 0; l < launches; ++l) {
+        if (geo.use && !build_maps(l, maps)) return cudaErrorInvalidValue;
+        geo.zbase = geo.use ? l : 0;
         Phase ph(MATE_PHASE_CHUNK_STATE, s);
-        ssd_chunk_state_tc_kernel<<<dim3(a.nh, a.nchunks, a.batch), kThreads, kStSmemBytes, s>>>(a, nsub);
+        ssd_chunk_state_tc_kernel<<<dim3(a.nh, a.nchunks, zdim), kThreads, kStSmemBytes, s>>>(a, nsub, maps.x, maps.b,
+                                                                                               geo);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
     {
         Phase ph(MATE_PHASE_STATE_PASS, s);
         ssd_state_chain_kernel<<<dim3(4096 / 8 / 256, a.nh * a.batch, 2), 256, 0, s>>>(a);
     }
-    {
+    for (int l = 0; l < launches; ++l) {
+        if (geo.use && !build_maps(l, maps)) return cudaErrorInvalidValue;
+        geo.zbase = geo.use ? l : 0;
         Phase ph(MATE_PHASE_CHUNK_OUT, s);
-        ssd_chunk_out_tc_kernel<<<dim3(a.nh, a.nchunks, a.batch), kThreads, kSmemBytes, s>>>(a, nsub);
+        ssd_chunk_out_tc_kernel<<<dim3(a.nh, a.nchunks, zdim), kThreads, kSmemBytes, s>>>(a, nsub, maps.x, maps.b,
+                                                                                         maps.c, geo);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

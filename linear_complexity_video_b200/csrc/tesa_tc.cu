@@ -26,13 +26,10 @@
 //      shared memory and stores those of queries in the grid as whole lines.
 // A window holds exactly one 128-token tile, so the softmax needs no online
 // rescaling.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
+#include "tmap.h"
 
 namespace mate {
 
@@ -368,35 +365,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
 // (batch element of a (T, H, W, nh, 128) bf16 tensor) -> 5-D map, box = 64 x 1 x Sw x Sw x Tw
 bool make_map(CUtensorMap *m, const void *base, const TesaArgs &a)
 {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t e = 2;
-    cuuint64_t dims[5] = {128, (cuuint64_t)a.nh, (cuuint64_t)a.W, (cuuint64_t)a.H, (cuuint64_t)a.T};
-    cuuint64_t strides[4] = {128 * e, (cuuint64_t)a.nh * 128 * e, (cuuint64_t)a.W * a.nh * 128 * e,
-                             (cuuint64_t)a.H * a.W * a.nh * 128 * e};
-    cuuint32_t box[5] = {64, 1, (cuuint32_t)a.Sw, (cuuint32_t)a.Sw, (cuuint32_t)a.Tw};
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    const uint64_t e = 2;
+    const uint64_t dims[5] = {128, (uint64_t)a.nh, (uint64_t)a.W, (uint64_t)a.H, (uint64_t)a.T};
+    const uint64_t strides[4] = {128 * e, (uint64_t)a.nh * 128 * e, (uint64_t)a.W * a.nh * 128 * e,
+                                 (uint64_t)a.H * a.W * a.nh * 128 * e};
+    const uint32_t box[5] = {64, 1, (uint32_t)a.Sw, (uint32_t)a.Sw, (uint32_t)a.Tw};
+    return tmap_bf16_5d(m, base, dims, strides, box);
 }
 
 }  // namespace
@@ -405,7 +382,7 @@ bool tesa_tc_supported(const TesaArgs &a)
 {
     return a.bf16 && a.d == 128 && a.Tw * a.Sw * a.Sw == 128 && a.Sw <= 128 && a.Tw <= 128 &&
            (size_t)a.nwt * a.nwh * a.nww * a.nh < ((size_t)1 << 31) &&
-           encode_fn() != nullptr;
+           tmap_available();
 }
 
 cudaError_t launch_tesa_tc(const TesaArgs &a, cudaStream_t s)
