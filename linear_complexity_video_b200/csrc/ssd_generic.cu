@@ -184,10 +184,13 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
 {
     constexpr int PR = P / RS;  // state rows of this CTA
     constexpr int PN = PR * NS;
-    constexpr int E = (PN + kThreads - 1) / kThreads;
-    constexpr int W = PR + NS + 1;                            // x rows | B | dt per position
-    constexpr int RT = W * 128 * 4 <= 40 * 1024 ? 128 : 32;   // positions per staged tile
-    __shared__ float vals[RT][W];
+    // thread t owns E consecutive elements t*E .. of the PR x NS block (one state
+    // row, adjacent columns): four per thread when they fill the CTA, else one
+    constexpr int E = (NS % 4 == 0 && PN >= 4 * kThreads) ? 4 : 1;
+    constexpr int NE = (PN + E * kThreads - 1) / (E * kThreads);  // element groups per thread
+    constexpr int W = (PR + NS + 1 + 3) & ~3;                     // x rows | B | decay, padded to 16 bytes
+    constexpr int RT = W * 128 * 4 <= 44 * 1024 ? 128 : 32;       // positions per staged tile
+    __shared__ __align__(16) float vals[RT][W];
     __shared__ int cells[RT];
     const int h = blockIdx.x, b = blockIdx.y, p0 = blockIdx.z * PR;
     const int grp = h / (a.nh / a.G);
@@ -195,9 +198,12 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
     const float Ah = a.A[h];
     const int L = 2 * a.Np;
     const float inv_box = 1.f / (float)(a.pt * a.ph * a.pw);
-    float s[E];
+    constexpr int WV = PR + NS + 1;  // staged values per position
+    float s[NE][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) s[e] = 0.f;
+    for (int u = 0; u < NE; ++u)
+#pragma unroll
+        for (int e = 0; e < E; ++e) s[u][e] = 0.f;
     for (int base = 0; base < L; base += RT) {
         __syncthreads();  // the previous tile is consumed
         for (int k = threadIdx.x; k < RT; k += blockDim.x) {
@@ -209,13 +215,13 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
         const int kmax = min(RT, L - base);
         // eight gathers in flight per thread
         constexpr int kU = 8;
-        for (int i0 = threadIdx.x; i0 < kmax * W; i0 += kU * blockDim.x) {
+        for (int i0 = threadIdx.x; i0 < kmax * WV; i0 += kU * blockDim.x) {
             const float *src[kU];
             float v[kU];
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
-                const int idx = min(i0 + u * (int)blockDim.x, kmax * W - 1);
-                const int k = idx / W, c = idx - k * W;
+                const int idx = min(i0 + u * (int)blockDim.x, kmax * WV - 1);
+                const int k = idx / WV, c = idx - k * WV;
                 const int col = c < PR ? h * P + p0 + c : (c < PR + NS ? CX + CD + grp * NS + (c - PR) : CX + h);
                 src[u] = a.pooled + ((size_t)b * a.pool_splits * a.Np + cells[k]) * CH + col;
                 v[u] = 0.f;
@@ -226,8 +232,8 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int idx = i0 + u * (int)blockDim.x;
-                if (idx < kmax * W) {
-                    const int k = idx / W, c = idx - k * W;
+                if (idx < kmax * WV) {
+                    const int k = idx / WV, c = idx - k * WV;
                     vals[k][c] = v[u] * inv_box;
                 }
             }
@@ -241,24 +247,34 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
             vals[k][PR + NS] = expf(dk * Ah);
         }
         __syncthreads();
-        // thread t owns the E consecutive elements t*E .. of the PR x NS block
-        // (one state row p, adjacent columns n)
         for (int k = 0; k < kmax; ++k) {
             const float dec = vals[k][PR + NS];
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const int idx = threadIdx.x * E + e;
-                if (idx < PN) {
-                    const int p = idx / NS, n = idx - p * NS;
-                    s[e] = fmaf(dec, s[e], vals[k][p] * vals[k][PR + n]);
+            for (int u = 0; u < NE; ++u) {
+                const int i0 = (threadIdx.x + u * kThreads) * E;
+                if (i0 < PN) {
+                    const int p = i0 / NS, n = i0 - p * NS;
+                    const float xp = vals[k][p];
+                    if (E == 4) {
+                        const float4 bv = *reinterpret_cast<const float4 *>(&vals[k][PR + n]);
+                        s[u][0] = fmaf(dec, s[u][0], xp * bv.x);
+                        s[u][1] = fmaf(dec, s[u][1], xp * bv.y);
+                        s[u][2] = fmaf(dec, s[u][2], xp * bv.z);
+                        s[u][3] = fmaf(dec, s[u][3], xp * bv.w);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < E; ++e) s[u][e] = fmaf(dec, s[u][e], xp * vals[k][PR + n + e]);
+                    }
                 }
             }
         }
     }
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int idx = threadIdx.x * E + e;
-        if (idx < PN) a.h_init[((size_t)b * a.nh + h) * (P * NS) + p0 * NS + idx] = s[e];
+    for (int u = 0; u < NE; ++u) {
+        const int i0 = (threadIdx.x + u * kThreads) * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            if (i0 + e < PN) a.h_init[((size_t)b * a.nh + h) * (P * NS) + p0 * NS + i0 + e] = s[u][e];
     }
 }
 
@@ -549,7 +565,7 @@ cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)
     }
     {
         Phase ph(MATE_PHASE_REVIEW_SCAN, s);
-        review_scan_kernel<64, 64, 8><<<dim3(a.nh, a.batch, 8), kThreads, 0, s>>>(a);
+        review_scan_kernel<64, 64, 4><<<dim3(a.nh, a.batch, 4), kThreads, 0, s>>>(a);
     }
     return cudaGetLastError();
 }

@@ -773,7 +773,7 @@ done:
 // runs in fp32, with the loads of kAhead chunks in flight ahead of it.
 // grid: (4096 / 8 / 256, nh * batch, 2 directions)
 // ---------------------------------------------------------------------------
-constexpr int kAhead = 8;
+constexpr int kAhead = 16;
 
 __global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
 {
