@@ -293,7 +293,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::mbar_init(ldbar, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
+        // TMA boxes need no grid offsets: sub-chunk 0's rows are requested first
+        if (geo.use) tma_rows(&mx, &mB, &mC, geo, sX, sB, nullptr, ldbar, h, grp, n0);
     }
+    if (geo.use) ++ld_issued;
     load_chunk_meta(a, b, h, n0, len, L, sgoff, sdt);
     tc::tc_fence_before();
     __syncthreads();
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         return *abort_flag == 0;
     };
     // x, B of sub-chunk 0 are in flight while the decay factors are prepared
-    issue_rows(sX, sB, nullptr, 0);
+    if (!geo.use) issue_rows(sX, sB, nullptr, 0);  // (the TMA batch is already in flight)
     sub_cumsums(sdt, scum, Ah, nsub, false, sred);
     // warp k: column factors of sub-chunk k around its midpoint r_k,
     //   gf[n] = exp(r_k - c_n) dt_n, gb[n] = exp(e_n - r_k) dt_n,
@@ -698,7 +701,10 @@ __global__ void __launch_bounds__(kThreads, 4)
         tc::mbar_init(ldbar, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
+        // TMA boxes need no grid offsets: sub-chunk 0's rows are requested first
+        if (geo.use) tma_rows(&mx, &mB, nullptr, geo, tX, tB, nullptr, ldbar, h, grp, n0);
     }
+    if (geo.use) ++ld_issued;
     load_chunk_meta(a, b, h, n0, len, L, sgoff, sdt);
     tc::tc_fence_before();
     __syncthreads();
@@ -709,8 +715,10 @@ __global__ void __launch_bounds__(kThreads, 4)
 
     for (int k = 0; k < nsub; ++k) {
         if (geo.use) {
-            if (tid == 0) tma_rows(&mx, &mB, nullptr, geo, tX, tB, nullptr, ldbar, h, grp, n0 + k * kSub);
-            ++ld_issued;
+            if (k > 0) {
+                if (tid == 0) tma_rows(&mx, &mB, nullptr, geo, tX, tB, nullptr, ldbar, h, grp, n0 + k * kSub);
+                ++ld_issued;
+            }
             if (tc::mbar_wait(ldbar, ld_phase & 1u, a.err))
                 ++ld_phase;
             else
