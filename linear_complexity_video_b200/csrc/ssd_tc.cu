@@ -492,27 +492,29 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
-        // row r of M: columns 64g .. 64g+63 of S times the decay factors -> tile g
+        // row r of M: 16-column groups g, g+2, g+4, g+6 of S times the decay factors.
+        // One group of each 32-column block, so every thread has exactly one group on
+        // the diagonal block of its warp's rows and the work is even across warps.
         {
             const float ff = __expf(ci - rmid), fb = __expf(rmid - ei);
             const int wq = warp & 3;  // this warp's rows are 32*wq .. 32*wq + 31
 #pragma unroll
-            for (int qp = 0; qp < 4; qp += 2) {
+            for (int m0 = 0; m0 < 4; m0 += 2) {
                 uint32_t raw2[2][16];  // two 16-column TMEM loads per wait
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp), raw2[0]);
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp + 16), raw2[1]);
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 16 * (2 * m0 + g)), raw2[0]);
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 16 * (2 * m0 + 2 + g)), raw2[1]);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int j0 = 64 * g + 16 * (qp + u);   // first of these 16 columns
+                    const int m = m0 + u;                    // 32-column block of this group
+                    const int j0 = 16 * (2 * m + g);         // first of its 16 columns
                     float sv[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sv[e] = __uint_as_float(raw2[u][e]);
-                    const int cc = j0 >> 5;             // 32-column block of these columns
-                    if (factored && cc != wq) {         // off the diagonal block: one direction only
+                    if (factored && m != wq) {               // off the diagonal block: one direction only
                         // left of every row of this warp: forward; right of every row: flipped
-                        const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? gf : gb) + j0);
-                        const float rf = cc < wq ? ff : fb;
+                        const float4 *fac = reinterpret_cast<const float4 *>((m < wq ? gf : gb) + j0);
+                        const float rf = m < wq ? ff : fb;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const float4 f4 = fac[q];
@@ -521,13 +523,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                             sv[4 * q + 2] *= rf * f4.z;
                             sv[4 * q + 3] *= rf * f4.w;
                         }
-                    } else if (factored) {              // the diagonal block
+                    } else if (factored) {                   // the diagonal block
+                        const float4 *f4p = reinterpret_cast<const float4 *>(gf + j0);
+                        const float4 *b4p = reinterpret_cast<const float4 *>(gb + j0);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int j = j0 + e;
-                            sv[e] *= (j <= r ? ff * gf[j] : 0.f) + (j >= r ? fb * gb[j] : 0.f);
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 f4 = f4p[q], b4 = b4p[q];
+                            const float fv[4] = {f4.x, f4.y, f4.z, f4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = j0 + 4 * q + e;
+                                sv[4 * q + e] *= (j <= r ? ff * fv[e] : 0.f) + (j >= r ? fb * bv[e] : 0.f);
+                            }
                         }
-                    } else {                            // decay range too wide: exact exponentials
+                    } else {                                 // decay range too wide: exact exponentials
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int j = j0 + e;
@@ -536,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                             sv[e] *= ((j <= r ? __expf(ci - cj) : 0.f) + (j >= r ? __expf(ej - ei) : 0.f)) * dj;
                         }
                     }
-                    uint8_t *tile = sM + g * kTile;
+                    uint8_t *tile = sM + (j0 >> 6) * kTile;
                     const int ch = (j0 & 63) >> 3;
                     *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch)) =
                         make_uint4(bf2(sv[0], sv[1]), bf2(sv[2], sv[3]), bf2(sv[4], sv[5]), bf2(sv[6], sv[7]));
