@@ -262,7 +262,10 @@ def run_mate(args, cfg, rank, world, dist):
             open_ev[phase] = ev
         else:
             phase_ms.setdefault(_lib.PHASES[phase], []).append(open_ev.pop(phase).elapsed_time(ev))
-    phase_avg = {k: sum(v) / len(v) for k, v in phase_ms.items()}
+    # a phase may launch once per batch element: per-step totals, and per-launch averages
+    phase_avg = {k: sum(v) / args.steps for k, v in phase_ms.items()}
+    phase_launch_avg = {k: sum(v) / len(v) for k, v in phase_ms.items()}
+    launches_per_step = {k: len(v) / args.steps for k, v in phase_ms.items()}
 
     # end to end through the public API with host buffers
     e2e = None
@@ -302,8 +305,8 @@ def run_mate(args, cfg, rank, world, dist):
         per_tok = algorithmic_bytes(cfg)
         # dominant kernel by time
         dom = max(phase_avg, key=lambda k: phase_avg[k])
-        dom_bytes = per_tok.get(dom, 0) * cfg.tokens
-        achieved = dom_bytes / (phase_avg[dom] / 1e3) / 1e9
+        dom_bytes = per_tok.get(dom, 0) * cfg.tokens / launches_per_step[dom]   # per launch
+        achieved = dom_bytes / (phase_launch_avg[dom] / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         value = job_throughput(cfg.tokens, world, ms_step)
         traffic = load_traffic(dom, cfg)
@@ -332,7 +335,8 @@ def run_mate(args, cfg, rank, world, dist):
             "phase_ms": {k: round(v, 4) for k, v in phase_avg.items()},
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_src},
+                         "algorithmic_bytes_per_launch": dom_bytes, "launches_per_step": launches_per_step[dom],
+                         "peak_source": peak_src},
             "gpu_launches": int(launches),
             "clocks": clocks,
             "e2e": e2e,
@@ -390,7 +394,8 @@ def time_config(cfg, mode, steps, warmup, seed=0):
         if not is_end:
             opened[ph] = ev
         else:
-            phases[_lib.PHASES[ph]] = round(opened.pop(ph).elapsed_time(ev), 4)
+            name = _lib.PHASES[ph]  # summed over the launches of one step
+            phases[name] = round(phases.get(name, 0.0) + opened.pop(ph).elapsed_time(ev), 4)
     if mate.mate_last_error() != 0:
         raise RuntimeError("device error word set")
     del d, out_ssd, out_att, ws
