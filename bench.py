@@ -213,8 +213,10 @@ def run_mate(args, cfg, rank, world, dist):
     marks = []
 
     def hook(phase, is_end, strm, user):
+        # recorded on the stream the library launches that phase on (a phase may run
+        # on the library's side stream)
         ev = torch.cuda.Event(enable_timing=True)
-        ev.record(stream)
+        ev.record(torch.cuda.ExternalStream(strm) if strm and strm != stream.cuda_stream else stream)
         marks.append((phase, is_end, ev))
 
     hook_c = _lib.PHASE_HOOK(hook)
@@ -370,8 +372,10 @@ def time_config(cfg, mode, steps, warmup, seed=0):
     marks = []
 
     def hook(phase, is_end, strm, user):
+        # recorded on the stream the library launches that phase on (a phase may run
+        # on the library's side stream)
         ev = torch.cuda.Event(enable_timing=True)
-        ev.record(stream)
+        ev.record(torch.cuda.ExternalStream(strm) if strm and strm != stream.cuda_stream else stream)
         marks.append((phase, is_end, ev))
 
     L = mate.load()
