@@ -55,6 +55,24 @@ def test_ssd_tc_ragged_batch2(mode):
     assert _run_ssd(cfg, inp, mode, (5, 3, 11), 256) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("mode", [0, 2])
+def test_ssd_tc_tma_rows_batch2(mode):
+    # 8x16x16 grid: every 128-position sub-chunk is a box of the grid in SR (16 w x 8 h)
+    # and TR (8 t x 16 w), so the rows come by TMA, one launch per batch element
+    cfg = BF16_SSD.with_(T=8, H=16, W=16, batch=2, nheads=3)
+    inp = workloads.generate(cfg, seed=6, parts=("ssd",))
+    assert _run_ssd(cfg, inp, mode, (2, 4, 4), 512) <= TOL["bf16"]
+
+
+def test_ssd_tc_tma_rows_past_the_end():
+    # 9x16x16 = 2304 tokens in SR order: boxes again, and the last 512-token chunk has two
+    # sub-chunks wholly past the sequence end, which the TMA fills with zeros
+    cfg = BF16_SSD.with_(T=9, H=16, W=16, nheads=3)
+    inp = workloads.generate(cfg, seed=7, parts=("ssd",))
+    assert _run_ssd(cfg, inp, 0, None, 512) <= TOL["bf16"]
+    assert _run_ssd(cfg, inp, 1, (3, 4, 4), 256) <= TOL["bf16"]
+
+
 def test_ssd_tc_groups():
     cfg = BF16_SSD.with_(T=4, H=8, W=16, nheads=4, ngroups=2)
     inp = workloads.generate(cfg, seed=3, parts=("ssd",))
