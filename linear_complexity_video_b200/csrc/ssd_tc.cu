@@ -30,7 +30,8 @@
 //              of S becomes row i of A = [ M | R_f C | R_b C ] (128 x 256) with
 //                  M_ij = S_ij dt_j (exp(c_i - c_j) [j <= i] + exp(e_j - e_i) [j >= i]),
 //                  R_f[i] = exp(c_i), R_b[i] = exp(c_end - e_i),
-//              and one accumulating MMA chain computes A . [ x ; h_f^T ; h_b^T ];
+//              and one accumulating MMA chain computes A . [ x ; h_f^T ; h_b^T ]
+//              (M as bf16 pairs in TMEM over S, read there as the A operand);
 //              the epilogue adds 2 D x and stores each row at its grid position.
 // The exponentials of M are factored around the sub-chunk midpoint r,
 // exp(c_i - c_j) = exp(c_i - r) exp(r - c_j), whenever the sub-chunk's decay
@@ -226,9 +227,11 @@ __device__ __forceinline__ bool mma_wait(uint64_t *bar, uint32_t &phase, int *er
 //   TMEM columns   0..127 : the K sub-chunk states, packed bf16 (32 columns each:
 //                           64 values of a state row per lane)
 //   TMEM columns 128..255 : phase 1 MMA result (64 cols), phase 3 S (128 cols),
-//                           then the output accumulator (64 cols)
+//                           then M as bf16 pairs (columns 0-31 and 96-127 of the
+//                           region) and the output accumulator (columns 32-95)
 //   shared memory         : x, B, C tiles of one sub-chunk; two 16 KB tiles for
-//                           U_f / U_b (phase 1) or M (phase 3); h_f, h_b operands.
+//                           U_f / U_b (phase 1) or the epilogue's staging (phase 3);
+//                           h_f, h_b operands.
 //                           In phase 3, R_f C overwrites the C tile and R_b C the
 //                           B tile once S = C B^T is done.
 // Loads overlap math: phase 1 double-buffers x, B in the {x, B} and {C, h}
@@ -492,29 +495,30 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
-        // row r of M: 16-column groups g, g+2, g+4, g+6 of S times the decay factors.
-        // One group of each 32-column block, so every thread has exactly one group on
-        // the diagonal block of its warp's rows and the work is even across warps.
+        // row r of M: S columns 64g .. 64g+63 times the decay factors, as bf16 pairs into
+        // TMEM columns 0..31 (g = 0) or 96..127 (g = 1) of R, over S columns this thread
+        // has already read; the output MMA reads M from there as its A operand.
         {
             const float ff = __expf(ci - rmid), fb = __expf(rmid - ei);
             const int wq = warp & 3;  // this warp's rows are 32*wq .. 32*wq + 31
+            uint32_t mp[2][16];       // the packed row half, 16 TMEM columns at a time
 #pragma unroll
-            for (int m0 = 0; m0 < 4; m0 += 2) {
+            for (int qp = 0; qp < 4; qp += 2) {
                 uint32_t raw2[2][16];  // two 16-column TMEM loads per wait
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 16 * (2 * m0 + g)), raw2[0]);
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 16 * (2 * m0 + 2 + g)), raw2[1]);
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp), raw2[0]);
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp + 16), raw2[1]);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int m = m0 + u;                    // 32-column block of this group
-                    const int j0 = 16 * (2 * m + g);         // first of its 16 columns
+                    const int j0 = 64 * g + 16 * (qp + u);   // first of these 16 columns
                     float sv[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sv[e] = __uint_as_float(raw2[u][e]);
-                    if (factored && m != wq) {               // off the diagonal block: one direction only
+                    const int cc = j0 >> 5;                  // 32-column block of these columns
+                    if (factored && cc != wq) {              // off the diagonal block: one direction only
                         // left of every row of this warp: forward; right of every row: flipped
-                        const float4 *fac = reinterpret_cast<const float4 *>((m < wq ? gf : gb) + j0);
-                        const float rf = m < wq ? ff : fb;
+                        const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? gf : gb) + j0);
+                        const float rf = cc < wq ? ff : fb;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const float4 f4 = fac[q];
@@ -545,14 +549,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                             sv[e] *= ((j <= r ? __expf(ci - cj) : 0.f) + (j >= r ? __expf(ej - ei) : 0.f)) * dj;
                         }
                     }
-                    uint8_t *tile = sM + (j0 >> 6) * kTile;
-                    const int ch = (j0 & 63) >> 3;
-                    *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch)) =
-                        make_uint4(bf2(sv[0], sv[1]), bf2(sv[2], sv[3]), bf2(sv[4], sv[5]), bf2(sv[6], sv[7]));
-                    *reinterpret_cast<uint4 *>(tile + tc::sw128(r, ch + 1)) =
-                        make_uint4(bf2(sv[8], sv[9]), bf2(sv[10], sv[11]), bf2(sv[12], sv[13]), bf2(sv[14], sv[15]));
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mp[qp >> 1][8 * u + e] = bf2(sv[2 * e], sv[2 * e + 1]);
                 }
             }
+            const uint32_t mcol = g ? 96u : 0u;
+            tc::tmem_st16(tc::tmem_addr(tR, lane_base, mcol), mp[0]);
+            tc::tmem_st16(tc::tmem_addr(tR, lane_base, mcol + 16), mp[1]);
+            tc::tmem_wait_st();
         }
         {
             // C row r, chunks 4g .. 4g+3 (this thread's own): R_f C over the C tile and
@@ -570,26 +574,28 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::tc_fence_before();
         __syncthreads();
 
-        // Acc = M x + (R_f C) h_f^T + (R_b C) h_b^T -> TMEM R columns 0..63
+        // Acc = M x + (R_f C) h_f^T + (R_b C) h_b^T -> TMEM R columns 32..95 (S there is
+        // consumed); M comes from TMEM (K-steps 0-3 at columns 0.., 4-7 at 96..)
+        const uint32_t tAcc = tR + 32;
         if (tid == 0) {
             tc::tc_fence_after();
             const uint32_t id_mx = tc::idesc_bf16(128, 64, 0, 1);
             const uint32_t id_ch = tc::idesc_bf16(128, 64, 0, 0);
-            const uint32_t m0 = tc::smem_u32(sM), x0 = tc::smem_u32(sX);
+            const uint32_t x0 = tc::smem_u32(sX);
             const uint32_t cf = tc::smem_u32(sC), cb = tc::smem_u32(sB);
             const uint32_t hf = tc::smem_u32(sHf), hb = tc::smem_u32(sHb);
 #pragma unroll
             for (int s2 = 0; s2 < 8; ++s2)
-                tc::mma_bf16(tR, tc::sdesc_sw128(m0 + (s2 >> 2) * kTile + (s2 & 3) * 32, 16, 1024),
-                             tc::sdesc_sw128(x0 + s2 * 2048, kTile, 1024), id_mx, s2 > 0);
+                tc::mma_bf16_tmem_a(tAcc, tR + (s2 < 4 ? 8 * s2 : 96 + 8 * (s2 - 4)),
+                                    tc::sdesc_sw128(x0 + s2 * 2048, kTile, 1024), id_mx, s2 > 0);
 #pragma unroll
             for (int s2 = 0; s2 < 4; ++s2)
-                tc::mma_bf16(tR, tc::sdesc_sw128(cf + s2 * 32, 16, 1024), tc::sdesc_sw128(hf + s2 * 32, 16, 1024), id_ch,
-                             true);
+                tc::mma_bf16(tAcc, tc::sdesc_sw128(cf + s2 * 32, 16, 1024), tc::sdesc_sw128(hf + s2 * 32, 16, 1024),
+                             id_ch, true);
 #pragma unroll
             for (int s2 = 0; s2 < 4; ++s2)
-                tc::mma_bf16(tR, tc::sdesc_sw128(cb + s2 * 32, 16, 1024), tc::sdesc_sw128(hb + s2 * 32, 16, 1024), id_ch,
-                             true);
+                tc::mma_bf16(tAcc, tc::sdesc_sw128(cb + s2 * 32, 16, 1024), tc::sdesc_sw128(hb + s2 * 32, 16, 1024),
+                             id_ch, true);
             tc::mma_commit(bar);
         }
         // this row's x (for the 2 D x term) to registers while the MMA runs (reads only)
@@ -612,8 +618,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         {
             uint8_t *stg = sM + warp * 2048;
             uint32_t acc2[2][16];
-            tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g), acc2[0]);
-            tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * g + 16), acc2[1]);
+            tc::tmem_ld16(tc::tmem_addr(tAcc, lane_base, 32 * g), acc2[0]);
+            tc::tmem_ld16(tc::tmem_addr(tAcc, lane_base, 32 * g + 16), acc2[1]);
             tc::tmem_wait_ld();
             const int lr = r & 31;  // this thread's row within the warp
 #pragma unroll
