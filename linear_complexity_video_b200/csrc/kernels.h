@@ -79,6 +79,8 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a);
 cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s);
 // the generic review pooling and prefix scan for bf16, head dim 64, d_state 64
 cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s);
+cudaError_t launch_review_pool_bf16_64(const SsdArgs &a, cudaStream_t s);  // its two halves
+cudaError_t launch_review_scan_bf16_64(const SsdArgs &a, cudaStream_t s);
 // generic CUDA-core TESA path
 cudaError_t launch_tesa_generic(const TesaArgs &a, cudaStream_t s);
 // tensor-core TESA path (bf16, head dim 128, 128-token windows)

@@ -549,6 +549,12 @@ cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s)
 
 cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)
 {
+    const cudaError_t e = launch_review_pool_bf16_64(a, s);
+    return e != cudaSuccess ? e : launch_review_scan_bf16_64(a, s);
+}
+
+cudaError_t launch_review_pool_bf16_64(const SsdArgs &a, cudaStream_t s)
+{
     const int CH = a.nh * a.P + a.nh + a.G * a.Ns;
     const bool vec = (a.nh * a.P) % 8 == 0 && (a.G * a.Ns) % 8 == 0 && a.nh % 4 == 0 &&
                      reinterpret_cast<uintptr_t>(a.dt) % 16 == 0;  // dt is read as float4
@@ -563,6 +569,11 @@ cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)
                 <<<dim3(a.Np, (CH + kThreads - 1) / kThreads, a.batch * a.pool_splits), kThreads, 0, s>>>(a);
         }
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_review_scan_bf16_64(const SsdArgs &a, cudaStream_t s)
+{
     {
         Phase ph(MATE_PHASE_REVIEW_SCAN, s);
         review_scan_kernel<64, 64, 4><<<dim3(a.nh, a.batch, 4), kThreads, 0, s>>>(a);

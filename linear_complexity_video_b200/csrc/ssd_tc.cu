@@ -683,6 +683,66 @@ constexpr uint32_t kStOffRed = kStOffGoff + kMaxChunk * 4;  // 8 floats
 constexpr uint32_t kStOffBar = kStOffRed + 64;
 constexpr uint32_t kStSmemBytes = kStOffBar + 64 + 1024;
 
+// Review pooling folded into chunk_state (RUN > 0): along the scan's fastest axis the
+// review box is RUN tokens long and RUN divides 128, so the rows of a sub-chunk come
+// in runs of RUN consecutive rows that share one pooling cell. Warp w builds rows
+// 32(w%4).. of the sub-chunk, columns 32g.. (g = w/4); its runs lie inside those rows,
+// so each warp sums its own runs from the x tile before it scales the tile in place:
+// a lane takes one (run, four columns) sum per RUN = 8 run, two per RUN = 4. The sums
+// of x (this head), dt and, for the group's first head, B stay in registers while the
+// lane's run in the next sub-chunk falls in the same cell (in time-major order the
+// sub-chunks of a chunk are neighbouring rows of one box); when the cell changes they
+// are added to the cell's totals with vector atomics. The separate pooling pass, which
+// would read x, dt and B once more, is then not needed.
+template <int RUN>
+struct RunSums {
+    static constexpr int NO = 8 / RUN;  // (run, four columns) sums per lane
+    float x[NO][4], b[NO][4], d[NO];
+    int cell[NO];  // -1: nothing held
+};
+
+// The lane's j-th run, counted in RUN-row runs from the warp's first row.
+__device__ __forceinline__ int lane_run(int j) { return ((threadIdx.x & 31) >> 3) + 4 * j; }
+
+// Sums over the rows of the lane's runs of four bf16 columns (c4 = column / 4) of an
+// SW128 tile. A warp reads rows of four runs at once; for RUN = 8 they alternate
+// between the two halves of the swizzled row, so each read is two bank wavefronts.
+template <int RUN>
+__device__ __forceinline__ void run_sums(const uint8_t *tile, int rbase, int c4, float (&out)[8 / RUN][4])
+{
+#pragma unroll
+    for (int j = 0; j < 8 / RUN; ++j) {
+        const int rl = lane_run(j);
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < RUN; ++i) {
+            const int r = rbase + RUN * rl + (RUN == 8 ? (i ^ (4 * (rl & 1))) : i);
+            const uint2 u = *reinterpret_cast<const uint2 *>(tile + tc::sw128(r, c4 >> 1) + (c4 & 1) * 8);
+            s[0] += __uint_as_float(u.x << 16);
+            s[1] += __uint_as_float(u.x & 0xffff0000u);
+            s[2] += __uint_as_float(u.y << 16);
+            s[3] += __uint_as_float(u.y & 0xffff0000u);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out[j][e] = s[e];
+    }
+}
+
+template <int RUN>
+__device__ __forceinline__ void run_flush(const SsdArgs &a, const RunSums<RUN> &acc, int j, int h, int grp,
+                                          int c4, bool with_d, bool with_b)
+{
+    if (acc.cell[j] < 0) return;
+    float *cell = a.pooled + (size_t)acc.cell[j] * (a.nh * a.P + a.nh + a.G * a.Ns);
+    atomicAdd(reinterpret_cast<float4 *>(cell + h * a.P + 4 * c4),
+              make_float4(acc.x[j][0], acc.x[j][1], acc.x[j][2], acc.x[j][3]));
+    if (with_d) atomicAdd(cell + a.nh * a.P + h, acc.d[j]);
+    if (with_b)
+        atomicAdd(reinterpret_cast<float4 *>(cell + a.nh * a.P + a.nh + grp * a.Ns + 4 * c4),
+                  make_float4(acc.b[j][0], acc.b[j][1], acc.b[j][2], acc.b[j][3]));
+}
+
+template <int RUN>
 __global__ void __launch_bounds__(kThreads, 4)
     ssd_chunk_state_tc_kernel(SsdArgs a, int nsub, const __grid_constant__ CUtensorMap mx,
                               const __grid_constant__ CUtensorMap mB, TmaRows geo)
@@ -709,6 +769,13 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int grp = h / (a.nh / a.G);
     const float Ah = a.A[h];
     uint32_t mma_phase = 0, ld_issued = 0, ld_phase = 0;  // TMA batches issued / completed
+    constexpr int RS = RUN > 0 ? RUN : 8;
+    RunSums<RS> runs;
+#pragma unroll
+    for (int j = 0; j < RunSums<RS>::NO; ++j) runs.cell[j] = -1;
+    const bool with_b = h % (a.nh / a.G) == 0;     // the group's first head pools B
+    const bool with_d = g == 0 && (tid & 7) == 0;  // one lane per run pools dt
+    const int c4 = 8 * g + (tid & 7), rbase = (warp & 3) * 32;
 
     if (warp == 0) tc::tmem_alloc(tmem_slot, 64);
     if (tid == 0) {
@@ -744,10 +811,45 @@ __global__ void __launch_bounds__(kThreads, 4)
         }
         __syncthreads();
         if (*abort_flag) goto done;
+        if constexpr (RUN > 0) {
+            // this warp's runs of the unscaled x; a run's cell from its first row's grid position
+            float xs[RunSums<RUN>::NO][4];
+            run_sums<RUN>(tX, rbase, c4, xs);
+#pragma unroll
+            for (int j = 0; j < RunSums<RUN>::NO; ++j) {
+                const int n0r = k * kSub + rbase + RUN * lane_run(j);
+                int cell = -1;
+                if (n0r < len) {
+                    const int gg = sgoff[n0r], hw = a.H * a.W;
+                    const int t = gg / hw, hh = (gg - t * hw) / a.W, ww = gg - t * hw - hh * a.W;
+                    cell = b * a.Np + ((t / a.pt) * a.Hp + hh / a.ph) * a.Wp + ww / a.pw;
+                }
+                if (cell != runs.cell[j]) {
+                    run_flush<RUN>(a, runs, j, h, grp, c4, with_d, with_b);
+                    runs.cell[j] = cell;
+                    runs.d[j] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) runs.x[j][e] = runs.b[j][e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) runs.x[j][e] += xs[j][e];
+            }
+            __syncwarp();  // the reads above come before this warp's in-place scaling
+        }
         {
             const int n = k * kSub + r;
             const float cj = scum[n], dj = sdt[n];
-            build_u(tX, tX, ub, r, g, __expf(cend - cj) * dj, __expf(cj - dj * Ah) * dj);
+            uint4 xv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const uint4 *>(tX + tc::sw128(r, 4 * g + q));
+            const __nv_bfloat162 f2 = __float2bfloat162_rn(__expf(cend - cj) * dj);
+            const __nv_bfloat162 b2 = __float2bfloat162_rn(__expf(cj - dj * Ah) * dj);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t off = tc::sw128(r, 4 * g + q);
+                *reinterpret_cast<uint4 *>(tX + off) = scale_chunk(xv[q], f2);
+                *reinterpret_cast<uint4 *>(ub + off) = scale_chunk(xv[q], b2);
+            }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -756,6 +858,27 @@ __global__ void __launch_bounds__(kThreads, 4)
             tc::tc_fence_after();
             mma_states(tmem, tc::smem_u32(tX), tc::smem_u32(tB), k > 0);
             tc::mma_commit(bar);
+        }
+        if constexpr (RUN > 0) {
+            // while the MMA runs: the runs' sums of dt and of B (which the MMA only reads)
+#pragma unroll
+            for (int j = 0; j < RunSums<RUN>::NO; ++j) {
+                if (with_d) {
+                    const float *d = sdt + k * kSub + rbase + RUN * lane_run(j);
+                    float sd = 0.f;
+#pragma unroll
+                    for (int i = 0; i < RUN; ++i) sd += d[i];
+                    runs.d[j] += sd;
+                }
+            }
+            if (with_b) {
+                float bs[RunSums<RUN>::NO][4];
+                run_sums<RUN>(tB, rbase, c4, bs);
+#pragma unroll
+                for (int j = 0; j < RunSums<RUN>::NO; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) runs.b[j][e] += bs[j][e];
+            }
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto done;
     }
@@ -777,6 +900,10 @@ __global__ void __launch_bounds__(kThreads, 4)
             *reinterpret_cast<uint4 *>(dst + 8 * q) = o;
         }
         if (tid == 0) a.alpha[((size_t)b * a.nh + h) * a.nchunks + c] = __expf(cend);
+        if constexpr (RUN > 0) {
+#pragma unroll
+            for (int j = 0; j < RunSums<RUN>::NO; ++j) run_flush<RUN>(a, runs, j, h, grp, c4, with_d, with_b);
+        }
     }
 done:
     tc::cp_async_wait_all();
@@ -861,11 +988,27 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(ssd_chunk_out_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ssd_chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kStSmemBytes);
-    if (e != cudaSuccess) return e;
+    // the review pooling folds into chunk_state when the review box is 4 or 8 tokens
+    // long along the scan's fastest axis and the channel blocks allow 16-byte atomics
+    int run = 0;
     if (a.review) {
-        e = launch_review_bf16_64(a, s);
+        const int r0 = a.mode == MATE_SCAN_SR ? a.pw : (a.mode == MATE_SCAN_SC ? a.ph : a.pt);
+        if ((r0 == 4 || r0 == 8) && a.nh % 4 == 0 && (a.G * a.Ns) % 4 == 0) run = r0;
+    }
+    auto st_kernel = run == 8 ? ssd_chunk_state_tc_kernel<8>
+                              : (run == 4 ? ssd_chunk_state_tc_kernel<4> : ssd_chunk_state_tc_kernel<0>);
+    e = cudaFuncSetAttribute(st_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStSmemBytes);
+    if (e != cudaSuccess) return e;
+    SsdArgs ar = a;  // the review scan reads one part of the box sums when they are pooled here
+    if (a.review) {
+        if (run) {
+            ar.pool_splits = 1;
+            Phase ph(MATE_PHASE_REVIEW_POOL, s);
+            e = cudaMemsetAsync(a.pooled, 0,
+                                (size_t)a.batch * a.Np * ((size_t)a.nh * a.P + a.nh + (size_t)a.G * a.Ns) * 4, s);
+        } else {
+            e = launch_review_pool_bf16_64(a, s);
+        }
         if (e != cudaSuccess) return e;
     }
     const int nsub = a.Q / kSub;
@@ -898,9 +1041,12 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
         if (geo.use && !build_maps(l, maps)) return cudaErrorInvalidValue;
         geo.zbase = geo.use ? l : 0;
         Phase ph(MATE_PHASE_CHUNK_STATE, s);
-        ssd_chunk_state_tc_kernel<<<dim3(a.nh, a.nchunks, zdim), kThreads, kStSmemBytes, s>>>(a, nsub, maps.x, maps.b,
-                                                                                               geo);
+        st_kernel<<<dim3(a.nh, a.nchunks, zdim), kThreads, kStSmemBytes, s>>>(a, nsub, maps.x, maps.b, geo);
         e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (a.review) {
+        e = launch_review_scan_bf16_64(ar, s);
         if (e != cudaSuccess) return e;
     }
     {

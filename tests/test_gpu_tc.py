@@ -73,6 +73,21 @@ def test_ssd_tc_tma_rows_past_the_end():
     assert _run_ssd(cfg, inp, 1, (3, 4, 4), 256) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_ssd_tc_review_runs(mode):
+    # review boxes 4 or 8 tokens long on the scan's fastest axis: runs of 4 or 8 rows of a
+    # sub-chunk share one box, and their sums are taken where the chunk states are; box
+    # rows by TMA (8x16x16), gathered rows (4x12x20), and two groups of two heads
+    cfg = BF16_SSD.with_(T=8, H=16, W=16, batch=2, nheads=4)
+    inp = workloads.generate(cfg, seed=8, parts=("ssd",))
+    assert _run_ssd(cfg, inp, mode, (8, 8, 8), 512) <= TOL["bf16"]
+    assert _run_ssd(cfg, inp, mode, (4, 4, 4), 256) <= TOL["bf16"]
+    cfg = BF16_SSD.with_(T=4, H=12, W=20, nheads=4, ngroups=2)
+    inp = workloads.generate(cfg, seed=9, parts=("ssd",))
+    assert _run_ssd(cfg, inp, mode, (4, 4, 4), 512) <= TOL["bf16"]
+    assert _run_ssd(cfg, inp, mode, (2, 4, 4), 384) <= TOL["bf16"]
+
+
 def test_ssd_tc_groups():
     cfg = BF16_SSD.with_(T=4, H=8, W=16, nheads=4, ngroups=2)
     inp = workloads.generate(cfg, seed=3, parts=("ssd",))
