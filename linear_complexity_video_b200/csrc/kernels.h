@@ -33,10 +33,15 @@ struct SsdArgs {
                              //   tensor-core path stores them as bf16)
     float *states_b;         // same for the flipped scan
     float *alpha;            // (batch, nh, nchunks): exp(A * sum of dt over the chunk)
-    float *h_init;           // (batch, nh, P, Ns): state after the review prefix
+    float *h_init;           // (kHinitParts, batch, nh, P, Ns): state after the review prefix;
+                             //   the tensor-core path writes it as parts over ranges of
+                             //   review cells that the state chain adds up, the CUDA-core
+                             //   path writes part 0 whole
     float *pooled;           // (batch, pool_splits, Np, nh*P + nh + G*Ns): partial box sums of x, dt, B
     int *err;                // device error word (MATE_ERR_* set by bounded waits)
 };
+
+constexpr int kHinitParts = 4;
 
 struct TesaArgs {
     const void *q;

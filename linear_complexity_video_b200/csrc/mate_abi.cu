@@ -187,7 +187,7 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a)
     l.alpha = off;
     off = align_up(off + (size_t)a.batch * a.nh * a.nchunks * sizeof(float));
     l.h_init = off;
-    if (a.review) off = align_up(off + (size_t)a.batch * a.nh * a.P * a.Ns * sizeof(float));
+    if (a.review) off = align_up(off + (size_t)kHinitParts * a.batch * a.nh * a.P * a.Ns * sizeof(float));
     l.pooled = off;
     if (a.review)
         off = align_up(off + (size_t)a.batch * a.pool_splits * a.Np *

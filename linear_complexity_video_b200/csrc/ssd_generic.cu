@@ -279,6 +279,143 @@ __global__ void __launch_bounds__(kThreads) review_scan_kernel(SsdArgs a)
 }
 
 // ---------------------------------------------------------------------------
+// review_hinit (P = Ns = 64): h_init without a sequential scan. Scanning the
+// prefix [R, flip(R)] (2 Np positions) from zero leaves
+//   h = sum_j exp(A * sum_{k>j} dt_k) * dt_j * x_j B_j^T,
+// and cell r of R sits at positions r and 2 Np - 1 - r. With d_r the cell's
+// pooled dt, P_r = sum_{r'<r} d_r' (the dt after position 2 Np - 1 - r) and
+// D = sum_r d_r (so 2D - P_r - d_r is the dt after position r):
+//   h = sum_r W_r x_r B_r^T,   W_r = d_r (exp(A P_r) + exp(A (2D - P_r - d_r))).
+// CTA z takes the z-th of kHinitParts ranges of cells and writes its part of
+// the sum to h_init part z; the state chain adds the parts. grid: (nh, batch,
+// kHinitParts)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 3) review_hinit_kernel(SsdArgs a)
+{
+    constexpr int P = 64, NS = 64, RT = 64;  // RT: cells per staged tile
+    constexpr int kDCap = 1024;              // pooled dt kept in shared memory up to this many cells
+    constexpr int kLd = RT * 32 / kThreads;  // 16-byte loads per thread per tile
+    __shared__ __align__(16) float xs[RT][P];
+    __shared__ __align__(16) float bs[RT][NS];
+    __shared__ float ws[RT];
+    __shared__ float dsm[kDCap];
+    __shared__ float red[2][kThreads / 32];
+    const int h = blockIdx.x, b = blockIdx.y, part = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = h / (a.nh / a.G);
+    const int CX = a.nh * P, CD = a.nh, CH = CX + CD + a.G * NS;
+    const float Ah = a.A[h];
+    const float inv_box = 1.f / (float)(a.pt * a.ph * a.pw);
+    const float *pb = a.pooled + (size_t)b * a.pool_splits * a.Np * CH;
+    const size_t split_stride = (size_t)a.Np * CH;
+    const bool vec = (CH & 3) == 0, dcache = a.Np <= kDCap;
+    int r0, r1;
+    split_range(a.Np, kHinitParts, part, r0, r1);
+    // pooled dt of the cell at position r of R (a box mean)
+    auto dbar = [&](int r) {
+        const float *src = pb + (size_t)rms_grid_offset(r, a.Tp, a.Hp, a.Wp, a.mode) * CH + CX + h;
+        float d = 0.f;
+        for (int sp = 0; sp < a.pool_splits; ++sp) d += src[sp * split_stride];
+        return d * inv_box;
+    };
+    // the loads of one tile's x rows (this head) and B rows (this group): box sums, four
+    // values a load, all of a thread's loads in flight at once
+    const float *src[kLd];
+    float4 v[kLd];
+    auto tile_loads = [&](int t0, int cnt) {
+#pragma unroll
+        for (int j = 0; j < kLd; ++j) {
+            const int i = tid + j * kThreads, k = min(i >> 5, cnt - 1), q = i & 31;
+            src[j] = pb + (size_t)rms_grid_offset(t0 + k, a.Tp, a.Hp, a.Wp, a.mode) * CH +
+                     (q < 16 ? h * P + 4 * q : CX + CD + grp * NS + 4 * (q - 16));
+            v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int sp = 0; sp < a.pool_splits; ++sp) {
+#pragma unroll
+            for (int j = 0; j < kLd; ++j) {
+                const float *s4 = src[j] + sp * split_stride;
+                const float4 u = vec ? *reinterpret_cast<const float4 *>(s4) : make_float4(s4[0], s4[1], s4[2], s4[3]);
+                v[j].x += u.x, v[j].y += u.y, v[j].z += u.z, v[j].w += u.w;
+            }
+        }
+    };
+    if (r0 < r1) tile_loads(r0, min(RT, r1 - r0));  // the first tile's rows load meanwhile
+    // D, and P_r at the first cell of this part
+    float dall = 0.f, dpre = 0.f;
+    for (int r = tid; r < a.Np; r += kThreads) {
+        const float d = dbar(r);
+        if (dcache) dsm[r] = d;
+        dall += d;
+        if (r < r0) dpre += d;
+    }
+    dall = warp_sum(dall);
+    dpre = warp_sum(dpre);
+    if (lane == 0) {
+        red[0][warp] = dall;
+        red[1][warp] = dpre;
+    }
+    __syncthreads();
+    float D2 = 0.f, carry = 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+        D2 += red[0][w];
+        carry += red[1][w];
+    }
+    D2 *= 2.f;
+    // thread: state rows 4 (t / 16) .. + 3, columns 4 (t % 16) .. + 3
+    const int p4 = (tid >> 4) * 4, n4 = (tid & 15) * 4;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int t0 = r0; t0 < r1; t0 += RT) {
+        const int cnt = min(RT, r1 - t0);
+        if (t0 != r0) {
+            __syncthreads();  // the previous tile is consumed
+            tile_loads(t0, cnt);
+        }
+#pragma unroll
+        for (int j = 0; j < kLd; ++j) {
+            const int i = tid + j * kThreads, k = i >> 5, q = i & 31;
+            if (k < cnt) *reinterpret_cast<float4 *>(q < 16 ? &xs[k][4 * q] : &bs[k][4 * (q - 16)]) = v[j];
+        }
+        if (warp == 0) {
+            // the tile's weights, two cells a lane, from an exclusive prefix of d over the tile;
+            // 1/box twice turns the x and B sums into means
+            const int k0 = 2 * lane;
+            float d0 = 0.f, d1 = 0.f;
+            if (k0 < cnt) d0 = dcache ? dsm[t0 + k0] : dbar(t0 + k0);
+            if (k0 + 1 < cnt) d1 = dcache ? dsm[t0 + k0 + 1] : dbar(t0 + k0 + 1);
+            const float incl = warp_inclusive_scan(d0 + d1);
+            const float p0 = carry + incl - (d0 + d1), p1 = p0 + d0;
+            const float sc = inv_box * inv_box;
+            if (k0 < cnt) ws[k0] = d0 * (expf(Ah * p0) + expf(Ah * (D2 - p0 - d0))) * sc;
+            if (k0 + 1 < cnt) ws[k0 + 1] = d1 * (expf(Ah * p1) + expf(Ah * (D2 - p1 - d1))) * sc;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        __syncthreads();
+        for (int k = 0; k < cnt; ++k) {
+            const float w = ws[k];
+            const float4 xv = *reinterpret_cast<const float4 *>(&xs[k][p4]);
+            const float4 bv = *reinterpret_cast<const float4 *>(&bs[k][n4]);
+            const float xw[4] = {xv.x * w, xv.y * w, xv.z * w, xv.w * w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[i][0] = fmaf(xw[i], bv.x, acc[i][0]);
+                acc[i][1] = fmaf(xw[i], bv.y, acc[i][1]);
+                acc[i][2] = fmaf(xw[i], bv.z, acc[i][2]);
+                acc[i][3] = fmaf(xw[i], bv.w, acc[i][3]);
+            }
+        }
+    }
+    float *dst = a.h_init + (((size_t)part * a.batch + b) * a.nh + h) * (P * NS) + p4 * NS + n4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4 *>(dst + i * NS) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+}
+
+// ---------------------------------------------------------------------------
 // chunk_state: chunk-local states from a zero start
 //   forward : sum_j exp(cum_end - cum_j) dt_j x_j B_j^T
 //   flipped : sum_j exp(excl_j) dt_j x_j B_j^T
@@ -576,7 +713,7 @@ cudaError_t launch_review_scan_bf16_64(const SsdArgs &a, cudaStream_t s)
 {
     {
         Phase ph(MATE_PHASE_REVIEW_SCAN, s);
-        review_scan_kernel<64, 64, 4><<<dim3(a.nh, a.batch, 4), kThreads, 0, s>>>(a);
+        review_hinit_kernel<<<dim3(a.nh, a.batch, kHinitParts), kThreads, 0, s>>>(a);
     }
     return cudaGetLastError();
 }

@@ -936,7 +936,16 @@ __global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
     const float *al = a.alpha + ((size_t)b * a.nh + h) * nc;
     float hv[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) hv[j] = a.review ? a.h_init[((size_t)b * a.nh + h) * 4096 + e8 + j] : 0.f;
+    for (int j = 0; j < 8; ++j) hv[j] = 0.f;
+    if (a.review) {  // h_init comes in parts over ranges of review cells
+        for (int part = 0; part < kHinitParts; ++part) {
+            const float4 *src = reinterpret_cast<const float4 *>(
+                a.h_init + (((size_t)part * a.batch + b) * a.nh + h) * 4096 + e8);
+            const float4 u = src[0], v = src[1];
+            hv[0] += u.x, hv[1] += u.y, hv[2] += u.z, hv[3] += u.w;
+            hv[4] += v.x, hv[5] += v.y, hv[6] += v.z, hv[7] += v.w;
+        }
+    }
     // one chain step: the stored chunk-local state becomes the entering state
     auto step_chunk = [&](int cidx, uint4 loc, float alpha) {
         uint4 o;
