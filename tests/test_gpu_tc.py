@@ -88,6 +88,17 @@ def test_ssd_tc_review_runs(mode):
     assert _run_ssd(cfg, inp, mode, (2, 4, 4), 384) <= TOL["bf16"]
 
 
+def test_ssd_tc_review_extremes():
+    # one review cell per token (2,048 cells: the cell weights do not fit in shared memory
+    # and every h_init part spans several tiles) and one cell for the whole grid (three of
+    # the four h_init parts are empty), with pooling runs of 8 along t in TC order
+    cfg = BF16_SSD.with_(T=8, H=16, W=16, nheads=4)
+    inp = workloads.generate(cfg, seed=10, parts=("ssd",))
+    assert _run_ssd(cfg, inp, 0, (1, 1, 1), 512) <= TOL["bf16"]
+    assert _run_ssd(cfg, inp, 0, (8, 16, 16), 512) <= TOL["bf16"]
+    assert _run_ssd(cfg, inp, 3, (8, 16, 16), 256) <= TOL["bf16"]
+
+
 def test_ssd_tc_groups():
     cfg = BF16_SSD.with_(T=4, H=8, W=16, nheads=4, ngroups=2)
     inp = workloads.generate(cfg, seed=3, parts=("ssd",))
