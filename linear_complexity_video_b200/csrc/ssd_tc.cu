@@ -519,13 +519,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                         // left of every row of this warp: forward; right of every row: flipped
                         const float4 *fac = reinterpret_cast<const float4 *>((cc < wq ? gf : gb) + j0);
                         const float rf = cc < wq ? ff : fb;
+                        const float2 rf2 = make_float2(rf, rf);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
+                        for (int q = 0; q < 4; ++q) {  // packed fp32 pairs
                             const float4 f4 = fac[q];
-                            sv[4 * q] *= rf * f4.x;
-                            sv[4 * q + 1] *= rf * f4.y;
-                            sv[4 * q + 2] *= rf * f4.z;
-                            sv[4 * q + 3] *= rf * f4.w;
+                            const float2 a = tc::mul_f32x2(make_float2(sv[4 * q], sv[4 * q + 1]),
+                                                           tc::mul_f32x2(rf2, make_float2(f4.x, f4.y)));
+                            const float2 c2 = tc::mul_f32x2(make_float2(sv[4 * q + 2], sv[4 * q + 3]),
+                                                            tc::mul_f32x2(rf2, make_float2(f4.z, f4.w)));
+                            sv[4 * q] = a.x, sv[4 * q + 1] = a.y, sv[4 * q + 2] = c2.x, sv[4 * q + 3] = c2.y;
                         }
                     } else if (factored) {                   // the diagonal block
                         const float4 *f4p = reinterpret_cast<const float4 *>(gf + j0);

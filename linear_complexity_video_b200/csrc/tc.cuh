@@ -200,6 +200,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// Two fp32 products in one packed instruction (round to nearest).
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b)
+{
+    uint64_t x, y, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+
 // 2^x by the hardware approximation (flush-to-zero; ex2(-inf) = +0).
 __device__ __forceinline__ float ex2_approx(float x)
 {
