@@ -442,9 +442,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tc::tmem_st16(tc::tmem_addr(tmem, lane_base, k * 32 + 16 * g), pk[u]);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
-                    const float2 f = tc::unpack_bf16(loc[u][q]);
-                    hv[2 * q] = fmaf(alpha, hv[2 * q], f.x);
-                    hv[2 * q + 1] = fmaf(alpha, hv[2 * q + 1], f.y);
+                    const float2 hn = tc::fma_f32x2(make_float2(alpha, alpha), make_float2(hv[2 * q], hv[2 * q + 1]),
+                                                    tc::unpack_bf16(loc[u][q]));
+                    hv[2 * q] = hn.x, hv[2 * q + 1] = hn.y;
                 }
             }
             tc::tmem_wait_st();
@@ -532,14 +532,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                     } else if (factored) {                   // the diagonal block
                         const float4 *f4p = reinterpret_cast<const float4 *>(gf + j0);
                         const float4 *b4p = reinterpret_cast<const float4 *>(gb + j0);
+                        const float2 ff2 = make_float2(ff, ff), fb2 = make_float2(fb, fb);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
+                        for (int q = 0; q < 4; ++q) {  // packed fp32 pairs
                             const float4 f4 = f4p[q], b4 = b4p[q];
-                            const float fv[4] = {f4.x, f4.y, f4.z, f4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                            const float2 tf[2] = {tc::mul_f32x2(ff2, make_float2(f4.x, f4.y)),
+                                                  tc::mul_f32x2(ff2, make_float2(f4.z, f4.w))};
+                            const float2 tb[2] = {tc::mul_f32x2(fb2, make_float2(b4.x, b4.y)),
+                                                  tc::mul_f32x2(fb2, make_float2(b4.z, b4.w))};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = j0 + 4 * q + e;
-                                sv[4 * q + e] *= (j <= r ? ff * fv[e] : 0.f) + (j >= r ? fb * bv[e] : 0.f);
+                            for (int e2 = 0; e2 < 2; ++e2) {
+                                const int j = j0 + 4 * q + 2 * e2;
+                                const float2 w = make_float2((j <= r ? tf[e2].x : 0.f) + (j >= r ? tb[e2].x : 0.f),
+                                                             (j + 1 <= r ? tf[e2].y : 0.f) + (j + 1 >= r ? tb[e2].y : 0.f));
+                                const float2 m = tc::mul_f32x2(make_float2(sv[4 * q + 2 * e2], sv[4 * q + 2 * e2 + 1]), w);
+                                sv[4 * q + 2 * e2] = m.x, sv[4 * q + 2 * e2 + 1] = m.y;
                             }
                         }
                     } else {                                 // decay range too wide: exact exponentials
@@ -631,9 +638,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint32_t o4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 xv = tc::unpack_bf16(xw[e]);
-                    o4[e] = bf2(fmaf(Dh2, xv.x, __uint_as_float(acc[2 * e])),
-                                fmaf(Dh2, xv.y, __uint_as_float(acc[2 * e + 1])));
+                    const float2 y2 = tc::fma_f32x2(make_float2(Dh2, Dh2), tc::unpack_bf16(xw[e]),
+                                                    make_float2(__uint_as_float(acc[2 * e]),
+                                                                __uint_as_float(acc[2 * e + 1])));
+                    o4[e] = bf2(y2.x, y2.y);
                 }
                 *reinterpret_cast<uint4 *>(stg + lr * 64 + ((q ^ ((lr >> 1) & 3)) << 4)) =
                     make_uint4(o4[0], o4[1], o4[2], o4[3]);
@@ -959,9 +967,9 @@ __global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
         const uint32_t w4[4] = {loc.x, loc.y, loc.z, loc.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float2 f = tc::unpack_bf16(w4[q]);
-            hv[2 * q] = fmaf(alpha, hv[2 * q], f.x);
-            hv[2 * q + 1] = fmaf(alpha, hv[2 * q + 1], f.y);
+            const float2 hn = tc::fma_f32x2(make_float2(alpha, alpha), make_float2(hv[2 * q], hv[2 * q + 1]),
+                                            tc::unpack_bf16(w4[q]));
+            hv[2 * q] = hn.x, hv[2 * q + 1] = hn.y;
         }
     };
     // visit chunks in chain order: forward 0 .. nc-1, flipped nc-1 .. 0

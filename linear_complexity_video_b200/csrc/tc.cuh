@@ -212,6 +212,19 @@ __device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b)
     return r;
 }
 
+// a * b + c on two fp32 pairs in one packed instruction (round to nearest).
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c)
+{
+    uint64_t x, y, z, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(z) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(x), "l"(y), "l"(z));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+
 // 2^x by the hardware approximation (flush-to-zero; ex2(-inf) = +0).
 __device__ __forceinline__ float ex2_approx(float x)
 {
