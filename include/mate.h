@@ -217,11 +217,13 @@ int mate_last_error(void *stream);
 
 /*
  * Phases of a call, reported to the phase hook below. Each phase is one
- * kernel launch.
+ * kernel launch, or (REVIEW_POOL when CHUNK_STATE takes the box sums, which
+ * it does when a review box is 4 or 8 tokens long on the scan's fastest axis
+ * on the tensor-core path) one clearing of the box-sum buffer.
  */
-#define MATE_PHASE_REVIEW_POOL 1 /* average-pool x, dt, B over the review boxes   */
-#define MATE_PHASE_REVIEW_SCAN 2 /* scan the review prefix -> its final state      */
-#define MATE_PHASE_CHUNK_STATE 3 /* chunk-local scan states                        */
+#define MATE_PHASE_REVIEW_POOL 1 /* box sums of x, dt, B over the review boxes     */
+#define MATE_PHASE_REVIEW_SCAN 2 /* the state the review prefix leaves (h_init)    */
+#define MATE_PHASE_CHUNK_STATE 3 /* chunk-local scan states (and box sums, above)  */
 #define MATE_PHASE_STATE_PASS 4  /* chain chunk states -> state entering each chunk */
 #define MATE_PHASE_CHUNK_OUT 5   /* outputs of every chunk, both directions         */
 #define MATE_PHASE_TESA 6        /* windowed attention                             */
