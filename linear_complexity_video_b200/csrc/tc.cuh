@@ -212,6 +212,18 @@ __device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b)
     return r;
 }
 
+// a + b on two fp32 pairs in one packed instruction (round to nearest).
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b)
+{
+    uint64_t x, y, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+
 // a * b + c on two fp32 pairs in one packed instruction (round to nearest).
 __device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c)
 {

@@ -281,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // P = 2^(S log2(e)/sqrt(d) - max') as bf16 pairs into TMEM columns
             // 16c .. 16c+15 (over S columns already read), and the row sum
             const float mxs = mx * p.scale_log2;
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-mxs, -mxs);
             float s8[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) s8[u] = 0.f;
@@ -288,9 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float e0 = tc::ex2_approx(fmaf(sv[c][2 * j], p.scale_log2, -mxs));
-                    const float e1 = tc::ex2_approx(fmaf(sv[c][2 * j + 1], p.scale_log2, -mxs));
+                for (int j = 0; j < 16; ++j) {  // exponent arguments as packed fp32 pairs
+                    const float2 t = tc::fma_f32x2(make_float2(sv[c][2 * j], sv[c][2 * j + 1]), sc2, nm2);
+                    const float e0 = tc::ex2_approx(t.x), e1 = tc::ex2_approx(t.y);
                     s8[(2 * j) & 7] += e0;
                     s8[(2 * j + 1) & 7] += e1;
                     pk[j] = tc::pack_bf16(e0, e1);
