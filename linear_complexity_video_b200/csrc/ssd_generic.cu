@@ -27,6 +27,7 @@
 //   chunk_out     intra-chunk quadratic term + entering states + D x
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace mate {
 
@@ -400,12 +401,13 @@ __global__ void __launch_bounds__(kThreads, 3) review_hinit_kernel(SsdArgs a)
             const float4 xv = *reinterpret_cast<const float4 *>(&xs[k][p4]);
             const float4 bv = *reinterpret_cast<const float4 *>(&bs[k][n4]);
             const float xw[4] = {xv.x * w, xv.y * w, xv.z * w, xv.w * w};
+            const float2 b01 = make_float2(bv.x, bv.y), b23 = make_float2(bv.z, bv.w);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[i][0] = fmaf(xw[i], bv.x, acc[i][0]);
-                acc[i][1] = fmaf(xw[i], bv.y, acc[i][1]);
-                acc[i][2] = fmaf(xw[i], bv.z, acc[i][2]);
-                acc[i][3] = fmaf(xw[i], bv.w, acc[i][3]);
+            for (int i = 0; i < 4; ++i) {  // packed fp32 pairs
+                const float2 x2 = make_float2(xw[i], xw[i]);
+                const float2 a01 = tc::fma_f32x2(x2, b01, make_float2(acc[i][0], acc[i][1]));
+                const float2 a23 = tc::fma_f32x2(x2, b23, make_float2(acc[i][2], acc[i][3]));
+                acc[i][0] = a01.x, acc[i][1] = a01.y, acc[i][2] = a23.x, acc[i][3] = a23.y;
             }
         }
     }

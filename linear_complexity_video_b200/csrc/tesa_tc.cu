@@ -324,10 +324,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < 8; ++q) {
                     const int u = q >> 2, c0 = (q & 3) * 8;
                     uint4 v;
-                    v.x = tc::pack_bf16(o[u][c0 + 0] * inv, o[u][c0 + 1] * inv);
-                    v.y = tc::pack_bf16(o[u][c0 + 2] * inv, o[u][c0 + 3] * inv);
-                    v.z = tc::pack_bf16(o[u][c0 + 4] * inv, o[u][c0 + 5] * inv);
-                    v.w = tc::pack_bf16(o[u][c0 + 6] * inv, o[u][c0 + 7] * inv);
+                    const float2 inv2 = make_float2(inv, inv);  // packed fp32 pairs
+                    const float2 o0 = tc::mul_f32x2(make_float2(o[u][c0 + 0], o[u][c0 + 1]), inv2);
+                    const float2 o1 = tc::mul_f32x2(make_float2(o[u][c0 + 2], o[u][c0 + 3]), inv2);
+                    const float2 o2 = tc::mul_f32x2(make_float2(o[u][c0 + 4], o[u][c0 + 5]), inv2);
+                    const float2 o3 = tc::mul_f32x2(make_float2(o[u][c0 + 6], o[u][c0 + 7]), inv2);
+                    v.x = tc::pack_bf16(o0.x, o0.y);
+                    v.y = tc::pack_bf16(o1.x, o1.y);
+                    v.z = tc::pack_bf16(o2.x, o2.y);
+                    v.w = tc::pack_bf16(o3.x, o3.y);
                     *reinterpret_cast<uint4 *>(stage + lane * 128 + ((q ^ (lane & 7)) << 4)) = v;
                 }
                 __syncwarp();
