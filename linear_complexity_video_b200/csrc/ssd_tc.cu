@@ -714,8 +714,8 @@ struct RunSums {
 // The lane's j-th run, counted in RUN-row runs from the warp's first row.
 __device__ __forceinline__ int lane_run(int j) { return ((threadIdx.x & 31) >> 3) + 4 * j; }
 
-// Sums over the rows of the lane's runs of four bf16 columns (c4 = column / 4) of an
-// SW128 tile. A warp reads rows of four runs at once; for RUN = 8 they alternate
+// Adds to out the sums over the rows of the lane's runs of four bf16 columns
+// (c4 = column / 4) of an SW128 tile. A warp reads rows of four runs at once; for RUN = 8 they alternate
 // between the two halves of the swizzled row, so each read is two bank wavefronts.
 template <int RUN>
 __device__ __forceinline__ void run_sums(const uint8_t *tile, int rbase, int c4, float (&out)[8 / RUN][4])
@@ -723,18 +723,15 @@ __device__ __forceinline__ void run_sums(const uint8_t *tile, int rbase, int c4,
 #pragma unroll
     for (int j = 0; j < 8 / RUN; ++j) {
         const int rl = lane_run(j);
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 s01 = make_float2(out[j][0], out[j][1]), s23 = make_float2(out[j][2], out[j][3]);
 #pragma unroll
-        for (int i = 0; i < RUN; ++i) {
+        for (int i = 0; i < RUN; ++i) {  // packed fp32 pairs
             const int r = rbase + RUN * rl + (RUN == 8 ? (i ^ (4 * (rl & 1))) : i);
             const uint2 u = *reinterpret_cast<const uint2 *>(tile + tc::sw128(r, c4 >> 1) + (c4 & 1) * 8);
-            s[0] += __uint_as_float(u.x << 16);
-            s[1] += __uint_as_float(u.x & 0xffff0000u);
-            s[2] += __uint_as_float(u.y << 16);
-            s[3] += __uint_as_float(u.y & 0xffff0000u);
+            s01 = tc::add_f32x2(s01, tc::unpack_bf16(u.x));
+            s23 = tc::add_f32x2(s23, tc::unpack_bf16(u.y));
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) out[j][e] = s[e];
+        out[j][0] = s01.x, out[j][1] = s01.y, out[j][2] = s23.x, out[j][3] = s23.y;
     }
 }
 
@@ -823,8 +820,6 @@ __global__ void __launch_bounds__(kThreads, 4)
         if (*abort_flag) goto done;
         if constexpr (RUN > 0) {
             // this warp's runs of the unscaled x; a run's cell from its first row's grid position
-            float xs[RunSums<RUN>::NO][4];
-            run_sums<RUN>(tX, rbase, c4, xs);
 #pragma unroll
             for (int j = 0; j < RunSums<RUN>::NO; ++j) {
                 const int n0r = k * kSub + rbase + RUN * lane_run(j);
@@ -841,9 +836,8 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) runs.x[j][e] = runs.b[j][e] = 0.f;
                 }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) runs.x[j][e] += xs[j][e];
             }
+            run_sums<RUN>(tX, rbase, c4, runs.x);
             __syncwarp();  // the reads above come before this warp's in-place scaling
         }
         {
@@ -881,14 +875,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                     runs.d[j] += sd;
                 }
             }
-            if (with_b) {
-                float bs[RunSums<RUN>::NO][4];
-                run_sums<RUN>(tB, rbase, c4, bs);
-#pragma unroll
-                for (int j = 0; j < RunSums<RUN>::NO; ++j)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) runs.b[j][e] += bs[j][e];
-            }
+            if (with_b) run_sums<RUN>(tB, rbase, c4, runs.b);
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto done;
     }
