@@ -212,6 +212,14 @@ __device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b)
     return r;
 }
 
+// max(a, b, c) in one instruction (a NaN operand is ignored, as by fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // a + b on two fp32 pairs in one packed instruction (round to nearest).
 __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b)
 {

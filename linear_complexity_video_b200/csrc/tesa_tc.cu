@@ -268,16 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!((kmask[c] >> j) & 1u)) sv[c][j] = -INFINITY;
             }
             // row maximum over eight independent chains
-            float m8[8];
+            float m8[8];  // two more values per chain per three-input max
 #pragma unroll
             for (int u = 0; u < 8; ++u) m8[u] = fmaxf(sv[0][u], sv[0][u + 8]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int i = 16; i < 128; i += 16)
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (c > 0 || j >= 16) m8[j & 7] = fmaxf(m8[j & 7], sv[c][j]);
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                for (int u = 0; u < 8; ++u)
+                    m8[u] = tc::fmax3(m8[u], sv[i >> 5][(i & 31) + u], sv[i >> 5][(i & 31) + u + 8]);
+            const float mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]),
+                                   tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
             // P = 2^(S log2(e)/sqrt(d) - max') as bf16 pairs into TMEM columns
             // 16c .. 16c+15 (over S columns already read), and the row sum
             const float mxs = mx * p.scale_log2;
