@@ -18,7 +18,17 @@
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller. The
  *     library allocates no device memory and keeps no state between calls,
- *     apart from one device-side error word (see mate_last_error).
+ *     with two exceptions that are part of its device image: one device-side
+ *     error word (see mate_last_error) and the fixed scratch array of
+ *     mate_bissd_fwd_noalloc (MATE_NOALLOC_SCRATCH_BYTES, below).
+ *   - Storage type decides which kernels run, with no fallback between them:
+ *     bf16 tensors run on the tensor-core (tcgen05) kernels, fp32 tensors on
+ *     the CUDA-core kernels. A bf16 call whose dims the tensor-core kernels
+ *     do not take returns MATE_ERR_UNSUPPORTED.
+ *   - The library caches, per device, the device addresses of its own device
+ *     variables. Destroying a device's primary context (cudaDeviceReset) is
+ *     detected through the context's unique id, and the addresses are looked
+ *     up again on the next call.
  *   - Tensors are dense and contiguous in grid order: for a batch element,
  *     token (t, h, w) sits at grid offset (t*H + h)*W + w, W fastest.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
@@ -91,11 +101,12 @@ typedef struct {
 } mate_attn_dims;
 
 /*
- * Workspace bytes mate_bissd_fwd needs for these dims (0 on bad arguments,
- * which mate_bissd_fwd then reports). The workspace holds per-chunk scan
- * states, chunk decays and, with review tokens, the pooled grid and the
- * state the review prefix leaves behind. Its contents on entry do not
- * matter.
+ * Workspace bytes mate_bissd_fwd needs for these dims (0 on bad or
+ * unsupported arguments, which mate_bissd_fwd then reports). The workspace
+ * holds per-chunk scan states of both directions (bf16 for bf16 storage,
+ * fp32 for fp32 storage), chunk decays and, with review tokens, the pooled
+ * grid and the state the review prefix leaves behind. Its contents on entry
+ * do not matter. It grows linearly with batch * T * H * W * nheads / chunk.
  */
 size_t mate_bissd_workspace_bytes(int T, int H, int W, const int review_pool[3], const mate_ssd_dims *d);
 
@@ -128,8 +139,17 @@ size_t mate_bissd_workspace_bytes(int T, int H, int W, const int review_pool[3],
  * x, B, C and out must be 16-byte aligned; dt, A, D 4-byte aligned.
  * workspace: >= mate_bissd_workspace_bytes(...) bytes of device memory,
  *   256-byte aligned, used only by the work this call enqueues.
- * Supported: headdim and dstate in {16, 32, 64}, chunk in [1, 256],
- *   nheads % ngroups == 0, T*H*W < 2^31.
+ * Supported (nheads % ngroups == 0 and T*H*W < 2^31 throughout):
+ *   bf16 storage (tensor-core kernels): headdim = dstate = 64, chunk a
+ *     multiple of 128 in [128, 512], directions = MATE_DIR_BI;
+ *   fp32 storage (CUDA-core kernels): headdim and dstate in {16, 32, 64},
+ *     chunk in [1, 256], any directions.
+ *   Anything else returns MATE_ERR_UNSUPPORTED before enqueueing work.
+ * Reproducibility: with review tokens on the tensor-core path, the review
+ *   box sums are accumulated with floating-point atomics, so the bits of
+ *   the result can differ from run to run (the differences are rounding
+ *   level, far inside the stated tolerance). Without review tokens, and on
+ *   the CUDA-core path, results are bitwise reproducible.
  * Returns MATE_OK, MATE_ERR_INVALID_ARG, MATE_ERR_UNSUPPORTED,
  *   MATE_ERR_WORKSPACE or MATE_ERR_CUDA.
  */
@@ -157,7 +177,8 @@ int mate_bissd_fwd(const void *x, const float *dt, const float *A, const void *B
  *   MATE_NOALLOC_SCRATCH_BYTES.
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture. The first call after the device's primary
+ *   context was destroyed and re-created looks it up again.
  * - All calls share the one array, which keeps the last call's contents.
  *   Calls whose work may overlap on the GPU (e.g. on unordered streams) race
  *   on it and must be serialised by the caller. Nothing needs clearing
@@ -185,7 +206,11 @@ int mate_bissd_fwd_noalloc(const void *x, const float *dt, const float *A, const
  *
  * Layouts: q, k, v, out : (batch, T, H, W, nheads, headdim), dtype,
  *   16-byte aligned.
- * Supported: headdim in {16, 32, 64, 128}, Tw*Sw*Sw <= 512.
+ * Supported:
+ *   bf16 storage (tensor-core kernel): headdim = 128, Tw*Sw*Sw = 128;
+ *   fp32 storage (CUDA-core kernel): headdim in {16, 32, 64, 128},
+ *     Tw*Sw*Sw <= 512.
+ *   Anything else returns MATE_ERR_UNSUPPORTED.
  * Returns MATE_OK, MATE_ERR_INVALID_ARG, MATE_ERR_UNSUPPORTED or
  *   MATE_ERR_CUDA.
  */

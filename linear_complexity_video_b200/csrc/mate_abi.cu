@@ -9,6 +9,7 @@
 
 #include "../../include/mate.h"
 #include "common.cuh"
+#include "devctx.h"
 #include "kernels.h"
 
 namespace mate {
@@ -23,18 +24,22 @@ mate_phase_hook g_hook = nullptr;
 void *g_hook_user = nullptr;
 }  // namespace
 
-// Device address of g_error_word on the current device (looked up once per device).
+// Device address of g_error_word in the current device's context, looked up once
+// per device and again after that device's context has been re-created.
 int *error_word_ptr()
 {
     static std::mutex mu;
     static int *addr[64] = {};
+    static unsigned long long ctx_of[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || ctx != ctx_of[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
         addr[dev] = static_cast<int *>(p);
+        ctx_of[dev] = ctx;
     }
     return addr[dev];
 }
@@ -119,11 +124,12 @@ int ssd_shape(int T, int H, int W, const int *pool, const mate_ssd_dims *d, int 
     return MATE_OK;
 }
 
-// 1 when the tensor-core path runs these dims, 0 when the CUDA-core path does,
-// -1 when neither can.
+// Which kernels run a bi-SSD call: bf16 storage runs on the tensor-core kernels
+// (1) and fp32 storage on the CUDA-core kernels (0); -1 when the kernels of that
+// storage type cannot take the dims. There is no fallback from one to the other.
 int ssd_path(const SsdArgs &a)
 {
-    if (ssd_tc_supported(a)) return 1;
+    if (a.bf16) return ssd_tc_supported(a) ? 1 : -1;
     const size_t smem = ((size_t)a.Q * (a.P + a.Ns) + 2 * a.P * a.Ns + 3 * (size_t)a.Q) * sizeof(float);
     if (a.Q > kMaxGenericChunk || smem > kMaxSmem) return -1;
     return 0;
@@ -179,11 +185,13 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a)
 {
     SsdWorkspace l;
     const size_t nstate = (size_t)a.batch * a.nh * a.nchunks * a.P * a.Ns;
+    // chunk states: bf16 on the tensor-core path (bf16 storage), fp32 on the CUDA-core path
+    const size_t state_bytes = a.bf16 ? 2 : 4;
     size_t off = 0;
     l.states_f = off;
-    off = align_up(off + nstate * sizeof(float));
+    off = align_up(off + nstate * state_bytes);
     l.states_b = off;
-    off = align_up(off + nstate * sizeof(float));
+    off = align_up(off + nstate * state_bytes);
     l.alpha = off;
     off = align_up(off + (size_t)a.batch * a.nh * a.nchunks * sizeof(float));
     l.h_init = off;
@@ -259,6 +267,8 @@ int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, i
     const size_t e = a.bf16 ? 2 : 4;
     const size_t maxm = (size_t)Tw * Sw * Sw;
     if (maxm > 512 || 2 * maxm * a.d * e + maxm * 4 > kMaxSmem) return MATE_ERR_UNSUPPORTED;
+    // bf16 storage runs on the tensor-core kernel, fp32 storage on the CUDA-core kernel
+    if (a.bf16 && !tesa_tc_supported(a)) return MATE_ERR_UNSUPPORTED;
     if (!q || !k || !v || !out) return MATE_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return MATE_ERR_INVALID_ARG;
     const size_t bytes = (size_t)a.batch * a.N * a.nh * a.d * e;
@@ -270,8 +280,8 @@ int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, i
     a.out = out;
     a.err = error_word_ptr();
     if (!a.err) return MATE_ERR_CUDA;
-    cudaError_t err = tesa_tc_supported(a) ? launch_tesa_tc(a, static_cast<cudaStream_t>(stream))
-                                           : launch_tesa_generic(a, static_cast<cudaStream_t>(stream));
+    cudaError_t err = a.bf16 ? launch_tesa_tc(a, static_cast<cudaStream_t>(stream))
+                             : launch_tesa_generic(a, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
 }
 

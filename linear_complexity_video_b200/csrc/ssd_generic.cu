@@ -1,5 +1,7 @@
 // Bidirectional Mamba2 (SSD) scan in Rotary Major Scan order with review
-// tokens: CUDA-core path for any supported head size, fp32 or bf16 storage.
+// tokens: CUDA-core path for fp32 storage and any supported head size (bf16
+// storage runs on the tensor-core kernels of ssd_tc.cu). The review pooling
+// kernels here also serve the tensor-core path.
 //
 // Method (paper review "LinGen ...", section 三, MA-Branch items 1-3): per
 // head, s_n = exp(dt_n A) s_{n-1} + dt_n x_n B_n^T and y_n = s_n C_n + D x_n,
@@ -683,7 +685,8 @@ cudaError_t dispatch_dims(const SsdArgs &a, cudaStream_t s)
 
 cudaError_t launch_ssd_generic(const SsdArgs &a, cudaStream_t s)
 {
-    return a.bf16 ? dispatch_dims<__nv_bfloat16>(a, s) : dispatch_dims<float>(a, s);
+    // fp32 storage only: bf16 calls run on the tensor-core kernels or are refused
+    return a.bf16 ? cudaErrorInvalidValue : dispatch_dims<float>(a, s);
 }
 
 cudaError_t launch_review_bf16_64(const SsdArgs &a, cudaStream_t s)

@@ -15,7 +15,8 @@
 //     returns MATE_ERR_WORKSPACE before enqueueing anything.
 //   - The first call on a device looks up the array's device address with
 //     cudaGetSymbolAddress (that device current); make that first call
-//     before any stream capture.
+//     before any stream capture. A call that finds the device's context
+//     re-created since then looks it up again.
 //   - All calls share the one array: calls whose work overlaps on the GPU
 //     (different streams, no ordering between them) race on it. The array
 //     keeps the last call's contents; the kernels write every scratch word
@@ -27,6 +28,7 @@
 #include <mutex>
 
 #include "../../include/mate.h"
+#include "devctx.h"
 
 namespace {
 
@@ -36,9 +38,11 @@ static __device__ __align__(256) unsigned char g_bissd_scratch[MATE_NOALLOC_SCRA
 
 std::mutex g_scratch_mu;
 void *g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of g_bissd_scratch on the current device (looked up once per
-// device), or nullptr with *rc set.
+// Device address of g_bissd_scratch in the current device's context (looked up
+// once per device, and again after that device's context has been re-created,
+// e.g. by cudaDeviceReset), or nullptr with *rc set.
 void *scratch_on_current_device(int *rc)
 {
     int dev = -1;
@@ -50,14 +54,16 @@ void *scratch_on_current_device(int *rc)
         *rc = MATE_ERR_UNSUPPORTED;
         return nullptr;
     }
+    const unsigned long long ctx = mate::current_context_id();
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    if (!g_scratch_addr[dev] || ctx != g_scratch_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_bissd_scratch) != cudaSuccess || !p) {
             *rc = MATE_ERR_CUDA;
             return nullptr;
         }
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     return g_scratch_addr[dev];
 }

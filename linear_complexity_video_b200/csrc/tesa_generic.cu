@@ -1,5 +1,5 @@
-// TEmporal Swin Attention, CUDA-core path for any supported head size and
-// window, fp32 or bf16 storage.
+// TEmporal Swin Attention, CUDA-core path for fp32 storage, any supported head
+// size and window (bf16 storage runs on the tensor-core kernel of tesa_tc.cu).
 //
 // Method (paper review "LinGen ...", section 三, TE-Branch): each token
 // attends only to the tokens of its Tw x Sw x Sw window; the window grid is
@@ -154,7 +154,8 @@ __global__ void rms_map_kernel(int T, int H, int W, int mode, int flip, int32_t 
 
 cudaError_t launch_tesa_generic(const TesaArgs &a, cudaStream_t s)
 {
-    return a.bf16 ? dispatch<__nv_bfloat16>(a, s) : dispatch<float>(a, s);
+    // fp32 storage only: bf16 calls run on the tensor-core kernel or are refused
+    return a.bf16 ? cudaErrorInvalidValue : dispatch<float>(a, s);
 }
 
 cudaError_t launch_tesa_map(const TesaArgs &a, int32_t *out, cudaStream_t s)

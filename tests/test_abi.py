@@ -114,3 +114,44 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(ImportError):
         _lib.load()
+
+
+def test_dispatch_by_storage_type():
+    """bf16 runs on the tensor-core kernels only and fp32 on the CUDA-core kernels
+    only: shapes the kernels of that storage type cannot take are refused on the
+    host, never sent to the other kernels."""
+    tc = dict(nheads=4, headdim=64, dstate=64, dtype=1)
+    ws = api.mate_bissd_workspace_bytes
+    for chunk in (128, 256, 384, 512):
+        assert ws(4, 8, 16, None, _dims(chunk=chunk, **tc)) > 0
+    for chunk in (64, 200, 640, 1024):                                   # not 128..512 in steps of 128
+        assert ws(4, 8, 16, None, _dims(chunk=chunk, **tc)) == 0
+    assert ws(4, 8, 16, None, _dims(chunk=256, **dict(tc, headdim=32))) == 0   # bf16 needs 64 x 64
+    assert ws(4, 8, 16, None, _dims(chunk=256, **dict(tc, dstate=16))) == 0
+    assert ws(4, 8, 16, None, _dims(chunk=256, directions=1, **tc)) == 0       # bf16: both directions only
+    assert ws(4, 8, 16, None, _dims(chunk=256)) > 0                             # fp32: CUDA-core kernels
+    assert ws(4, 8, 16, None, _dims(chunk=256, directions=1)) > 0
+    assert ws(4, 8, 16, None, _dims(chunk=384)) == 0                            # fp32: chunk <= 256
+    L = mate.load()
+    assert _call_bissd(L, dims=_dims(chunk=256, **dict(tc, headdim=32))) == _lib.MATE_ERR_UNSUPPORTED
+    assert _call_bissd(L, dims=_dims(chunk=200, **tc)) == _lib.MATE_ERR_UNSUPPORTED
+    # bf16 attention: head dim 128 and 128-token windows only
+    p = ctypes.c_void_p(1 << 20)
+    o = ctypes.c_void_p(1 << 32)
+    sh = (ctypes.c_int * 3)(0, 0, 0)
+    for dims, Tw, Sw in (((1, 2, 64, 1), 2, 8), ((1, 2, 128, 1), 2, 4)):
+        d = _lib.mate_attn_dims(*dims)
+        assert L.tesa_fwd(p, p, p, 4, 8, 8, Tw, Sw, sh, o, ctypes.byref(d), None) == _lib.MATE_ERR_UNSUPPORTED
+
+
+def test_workspace_layout_by_storage_type():
+    """Chunk states take 2 bytes per element for bf16 storage and 4 for fp32."""
+    def expected(nchunks, nh, state_bytes):
+        align = lambda v: (v + 255) // 256 * 256
+        states = align(nchunks * nh * 64 * 64 * state_bytes)
+        return 2 * states + align(nchunks * nh * 4)
+    # 2,048 tokens, chunk 256 -> 8 chunks, 4 heads of 64 x 64, no review tokens
+    assert api.mate_bissd_workspace_bytes(8, 16, 16, None, _dims(nheads=4, headdim=64, dstate=64, chunk=256,
+                                                                 dtype=1)) == expected(8, 4, 2)
+    assert api.mate_bissd_workspace_bytes(8, 16, 16, None, _dims(nheads=4, headdim=64, dstate=64, chunk=256,
+                                                                 dtype=0)) == expected(8, 4, 4)
