@@ -4,10 +4,11 @@ synthetic latent grid.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl mate|reference]
 
-Prints one JSON line (rank 0). With N > 1 (torchrun, one rank per GPU) every
-rank processes its own batch element drawn with its own seed: the path has
-no exchange step, so this is weak scaling with no collective on the data
-path; the NCCL group only carries the barrier and the max-over-ranks time.
+Prints one JSON line (rank 0). With N > 1 (torchrun, one rank per GPU; a
+plain `python bench.py --gpus N` starts the N ranks itself) every rank
+processes its own batch element drawn with its own seed: the path has no
+exchange step, so this is weak scaling with no collective on the data path;
+the NCCL group only carries the barrier and the max-over-ranks time.
 
 --impl reference times the fp64 CPU oracle (the only other code this script
 may run) on the same workload, one bounded sample per step.
@@ -56,6 +57,24 @@ def algorithmic_bytes(cfg):
     }
     per_tok["bissd"] = 2 * x + dt + 2 * bc                   # the MA-branch as one op
     return per_tok
+
+
+def mma_flops(cfg):
+    """Tensor-core flops per token of each kernel, as the kernels issue them
+    (bf16 path: 128-token sub-chunks, both scan directions).
+    chunk_state: one MMA [U_f^T; U_b^T] (2P x 128) . B (128 x Ns) per sub-chunk.
+    chunk_out: that MMA again, S = C B^T (128 x 128 x Ns), M x (128 x P x 128)
+    and R_f C h_f^T + R_b C h_b^T (2 x 128 x P x Ns) per sub-chunk.
+    tesa: Q K^T and P V over every key of the token's window."""
+    P, Ns, nh = cfg.headdim, cfg.dstate, cfg.nheads
+    q = 128
+    state = 2 * (2 * P) * Ns
+    out = state + 2 * q * Ns + 2 * q * P + 2 * (2 * P * Ns)
+    win = cfg.Tw * cfg.Sw * cfg.Sw
+    f = {"review_pool": 0, "chunk_state": nh * state, "state_pass": 0, "chunk_out": nh * out,
+         "tesa": cfg.attn_heads * 4 * cfg.attn_dim * win}
+    f["bissd"] = f["chunk_state"] + f["chunk_out"]
+    return f
 
 
 def load_peaks():
@@ -312,6 +331,14 @@ def run_mate(args, cfg, rank, world, dist):
         dom_bytes = per_tok.get(dom, 0) * cfg.tokens / launches_per_step[dom]   # per launch
         achieved = dom_bytes / (phase_launch_avg[dom] / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
+        tc_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        flops = mma_flops(cfg)
+        dom_flops = flops.get(dom, 0) * cfg.tokens / launches_per_step[dom]
+        tensor_tflops = dom_flops / (phase_launch_avg[dom] / 1e3) / 1e12
+        path_bytes = (per_tok["bissd"] + per_tok["tesa"]) * cfg.tokens
+        path_flops = (flops["bissd"] + flops["tesa"]) * cfg.tokens
+        path_gbs = path_bytes / (ms_step / 1e3) / 1e9
+        path_tflops = path_flops / (ms_step / 1e3) / 1e12
         value = job_throughput(cfg.tokens, world, ms_step)
         traffic = load_traffic(dom, cfg)
         result = {
@@ -340,7 +367,12 @@ def run_mate(args, cfg, rank, world, dist):
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": dom_bytes, "launches_per_step": launches_per_step[dom],
-                         "peak_source": peak_src},
+                         "peak_source": peak_src,
+                         "tensor_tflops": tensor_tflops, "tensor_peak": tc_peak,
+                         "tensor_frac": tensor_tflops / tc_peak, "mma_flops_per_launch": dom_flops,
+                         "path_frac": path_gbs / peak, "path_gbs": path_gbs,
+                         "path_tensor_frac": path_tflops / tc_peak,
+                         "path_bytes_per_step": path_bytes, "path_mma_flops_per_step": path_flops},
             "gpu_launches": int(launches),
             "clocks": clocks,
             "e2e": e2e,
@@ -510,6 +542,47 @@ def run_reference(args, cfg):
     }
 
 
+def spawn_ranks(args) -> int:
+    """--gpus N without an outside launcher: start N ranks of this script on
+    this node through torch.distributed.run (one process per GPU) and return
+    its exit status. The GPU arm needs N visible devices."""
+    import socket
+
+    n = args.gpus
+    if args.impl == "mate":
+        import torch
+
+        have = torch.cuda.device_count()
+        if have < n:
+            print(f"bench.py: --gpus {n} needs {n} CUDA devices, {have} visible", file=sys.stderr)
+            return 2
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+def join_ranks(rank: int, world: int) -> int:
+    """Reference arm under N ranks: every rank checks in over a CPU (gloo)
+    group, then all but rank 0 leave; rank 0 alone times the oracle.
+    Returns the number of ranks that checked in."""
+    if world <= 1:
+        return 1
+    import datetime
+
+    import torch.distributed as tdist
+
+    tdist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    seen = [None] * world
+    tdist.all_gather_object(seen, rank)
+    tdist.destroy_process_group()
+    if rank != 0:
+        print(f"bench.py rank {rank}/{world}: reference arm runs on rank 0 only", file=sys.stderr, flush=True)
+    return len(set(seen))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -531,12 +604,21 @@ def main():
     cfg = workloads.CONFIGS[args.config]
     if args.chunk:
         cfg = cfg.with_(chunk=args.chunk)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(spawn_ranks(args))
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
+    if world != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
 
     if args.impl == "reference":
+        joined = join_ranks(rank, world)
         if rank == 0:
-            print(json.dumps(run_reference(args, cfg)), flush=True)
+            res = run_reference(args, cfg)
+            res["n_gpus"] = world
+            if world > 1:
+                res["ranks_joined"] = joined
+            print(json.dumps(res), flush=True)
         return
     if args.report:
         run_report(args)

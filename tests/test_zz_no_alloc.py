@@ -38,7 +38,9 @@ def _noalloc_call(L, dev, cfg, mode, pool, out):
                                     cfg.T, cfg.H, cfg.W, mode, pool_arr, p(out), ctypes.byref(dims), stream)
 
 
-@pytest.mark.parametrize("name,heads,mode", [("tiny", None, 2), ("512p-17s", 4, 3)])
+# 256p-17s at all 80 heads needs 20 MiB with its states sized at bf16 (the
+# tensor-core path's storage); sized at fp32 it would not fit in 32 MiB.
+@pytest.mark.parametrize("name,heads,mode", [("tiny", None, 2), ("512p-17s", 4, 3), ("256p-17s", None, 0)])
 def test_noalloc_matches_workspace_entry_point(name, heads, mode):
     cfg = workloads.CONFIGS[name]
     if heads is not None:
@@ -60,7 +62,7 @@ def test_noalloc_matches_workspace_entry_point(name, heads, mode):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    cfg = workloads.CONFIGS["256p-17s"]
+    cfg = workloads.CONFIGS["512p-17s"].with_(review=None)
     dims = api.ssd_dims(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, cfg.ngroups, cfg.chunk, cfg.torch_dtype)
     assert api.mate_bissd_workspace_bytes(cfg.T, cfg.H, cfg.W, cfg.review, dims) > _lib.NOALLOC_SCRATCH_BYTES
     dev = to_dev(workloads.generate(cfg.with_(T=1), parts=("ssd",)))  # pointers only; nothing may be written
