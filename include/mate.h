@@ -104,8 +104,10 @@ typedef struct {
  * Workspace bytes mate_bissd_fwd needs for these dims (0 on bad or
  * unsupported arguments, which mate_bissd_fwd then reports). The workspace
  * holds per-chunk scan states of both directions (bf16 for bf16 storage,
- * fp32 for fp32 storage), chunk decays and, with review tokens, the pooled
- * grid and the state the review prefix leaves behind. Its contents on entry
+ * fp32 for fp32 storage), chunk decays, for bf16 storage dt in scan order
+ * (fp32, one value per head and scan position, padded to whole chunks) and,
+ * with review tokens, the pooled grid and the state the review prefix
+ * leaves behind. Its contents on entry
  * do not matter. It grows linearly with batch * T * H * W * nheads / chunk.
  */
 size_t mate_bissd_workspace_bytes(int T, int H, int W, const int review_pool[3], const mate_ssd_dims *d);

@@ -38,6 +38,8 @@ struct SsdArgs {
                              //   review cells that the state chain adds up, the CUDA-core
                              //   path writes part 0 whole
     float *pooled;           // (batch, pool_splits, Np, nh*P + nh + G*Ns): partial box sums of x, dt, B
+    float *dt_scan;          // (batch, nh, nchunks * Q): dt in scan order, zero past the sequence
+                             //   end; written by the tensor-core chunk_state for chunk_out
     int *err;                // device error word (MATE_ERR_* set by bounded waits)
 };
 
@@ -76,7 +78,7 @@ struct Phase {
 
 // Workspace layout of a bi-SSD call; offsets in bytes from the base pointer.
 struct SsdWorkspace {
-    size_t states_f, states_b, alpha, h_init, pooled, total;
+    size_t states_f, states_b, alpha, h_init, pooled, dt_scan, total;
 };
 SsdWorkspace ssd_workspace_layout(const SsdArgs &a);
 

@@ -144,6 +144,7 @@ void carve(SsdArgs &a, void *ws)
     a.alpha = reinterpret_cast<float *>(base + l.alpha);
     a.h_init = a.review ? reinterpret_cast<float *>(base + l.h_init) : nullptr;
     a.pooled = a.review ? reinterpret_cast<float *>(base + l.pooled) : nullptr;
+    a.dt_scan = a.bf16 ? reinterpret_cast<float *>(base + l.dt_scan) : nullptr;
 }
 
 int attn_shape(int T, int H, int W, int Tw, int Sw, const int *shift, const mate_attn_dims *d, TesaArgs &a)
@@ -200,6 +201,9 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a)
     if (a.review)
         off = align_up(off + (size_t)a.batch * a.pool_splits * a.Np *
                                  ((size_t)a.nh * a.P + a.nh + (size_t)a.G * a.Ns) * sizeof(float));
+    // tensor-core path: dt of every chunk in scan order (chunk_state -> chunk_out)
+    l.dt_scan = off;
+    if (a.bf16) off = align_up(off + (size_t)a.batch * a.nh * a.nchunks * a.Q * sizeof(float));
     l.total = off;
     return l;
 }

@@ -140,6 +140,12 @@ __device__ __forceinline__ void load_chunk_meta(const SsdArgs &a, int b, int h, 
     }
 }
 
+// Grid offsets of the chunk's L positions (0 past the sequence end).
+__device__ __forceinline__ void chunk_offsets(const SsdArgs &a, int n0, int len, int L, int *goff)
+{
+    for (int n = threadIdx.x; n < L; n += kThreads) goff[n] = n < len ? rms_grid_offset(n0 + n, a.T, a.H, a.W, a.mode) : 0;
+}
+
 // Inclusive cumulative sums of A*dt within each 128-token sub-chunk (warp w
 // scans sub-chunk w); with `chunk_level`, continued across sub-chunks.
 __device__ __forceinline__ void sub_cumsums(const float *dt, float *cum, float Ah, int nsub, bool chunk_level,
@@ -244,15 +250,16 @@ constexpr uint32_t kOffB = kTile;
 constexpr uint32_t kOffC = 2 * kTile;
 constexpr uint32_t kOffM = 3 * kTile;       // 2 tiles: U_f, U_b / M0, M1
 constexpr uint32_t kOffH = 5 * kTile;       // h_f (8 KB) then h_b (8 KB)
-constexpr uint32_t kOffDt = 6 * kTile;
-constexpr uint32_t kOffCum = kOffDt + kMaxChunk * 4;
+constexpr uint32_t kOffDt = 6 * kTile;                // 2 x dt[512]: this item's, the next item's
+constexpr uint32_t kOffCum = kOffDt + 2 * kMaxChunk * 4;
 constexpr uint32_t kOffGoff = kOffCum + kMaxChunk * 4;
 constexpr uint32_t kOffGf = kOffGoff + kMaxChunk * 4;
 constexpr uint32_t kOffGb = kOffGf + kMaxChunk * 4;
 constexpr uint32_t kOffRed = kOffGb + kMaxChunk * 4;  // 8 floats
 constexpr uint32_t kOffFlag = kOffRed + 32;           // kMaxSubs ints: sub-chunk takes the factored exps
 constexpr uint32_t kOffBar = kOffRed + 64;
-constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;
+constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;  // bar, TMEM slot, abort flag, ldbar, dtbar
+static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "chunk_out: two CTAs per SM");
 
 constexpr uint32_t kColR = 128;   // scratch region after the packed state slots
 constexpr uint32_t kTmemCols = 256;
@@ -261,14 +268,15 @@ __device__ __forceinline__ uint32_t bf2(float lo, float hi) { return tc::pack_bf
 
 __global__ void __launch_bounds__(kThreads, 2)
     ssd_chunk_out_tc_kernel(SsdArgs a, int nsub, const __grid_constant__ CUtensorMap mx,
-                            const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC, TmaRows geo)
+                            const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
+                            const __grid_constant__ CUtensorMap mO, TmaRows geo, int nitems)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     uint8_t *sX = base + kOffX, *sB = base + kOffB, *sC = base + kOffC, *sM = base + kOffM;
     uint8_t *sHf = base + kOffH, *sHb = base + kOffH + 8192;
-    float *sdt = reinterpret_cast<float *>(base + kOffDt);
+    float *sdt_buf = reinterpret_cast<float *>(base + kOffDt);
     float *scum = reinterpret_cast<float *>(base + kOffCum);
     int *sgoff = reinterpret_cast<int *>(base + kOffGoff);
     float *sgf = reinterpret_cast<float *>(base + kOffGf);
@@ -279,28 +287,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffBar + 8);
     int *abort_flag = reinterpret_cast<int *>(base + kOffBar + 12);
     uint64_t *ldbar = reinterpret_cast<uint64_t *>(base + kOffBar + 16);  // TMA row loads
+    uint64_t *dtbar = reinterpret_cast<uint64_t *>(base + kOffBar + 24);  // dt of an item
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r = tid & (kSub - 1), g = tid >> 7;   // row / TMEM lane, column half
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-    const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z + geo.zbase;
     const int L = nsub * kSub;
-    const int n0 = c * L, len = min(L, a.N - n0);
-    const int grp = h / (a.nh / a.G);
-    const float Ah = a.A[h], Dh2 = 2.f * a.D[h];
-    uint32_t mma_phase = 0, ld_issued = 0, ld_phase = 0;  // TMA batches issued / completed
+    uint32_t ld_issued = 0, ld_phase = 0;  // TMA batches issued / completed
+    uint32_t dt_issued = 0, dt_phase = 0;  // dt loads issued / completed
+    uint32_t mma_phase = 0;                // MMA completions on bar
+    // the work item in hand: head h of chunk c of batch element b (heads fastest)
+    int h = 0, c = 0, b = 0, n0 = 0, len = 0, grp = 0;
+    float Ah = 0.f, Dh2 = 0.f;
+    // dt of item `it` (written in scan order by chunk_state) into dt buffer `buf`,
+    // completing on dtbar; issued by one thread
+    auto issue_dt = [&](int it, int buf) {
+        const int ih = it % a.nh, ic = (it / a.nh) % a.nchunks, ib = it / (a.nh * a.nchunks) + geo.zbase;
+        tc::mbar_expect_tx(dtbar, (uint32_t)L * 4u);
+        tc::bulk_load(sdt_buf + buf * kMaxChunk, a.dt_scan + (((size_t)ib * a.nh + ih) * a.nchunks + ic) * L,
+                      (uint32_t)L * 4u, dtbar);
+    };
 
     if (warp == 0) tc::tmem_alloc(tmem_slot, kTmemCols);
     if (tid == 0) {
         tc::mbar_init(bar, 1);
         tc::mbar_init(ldbar, 1);
+        tc::mbar_init(dtbar, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
-        // TMA boxes need no grid offsets: sub-chunk 0's rows are requested first
-        if (geo.use) tma_rows(&mx, &mB, &mC, geo, sX, sB, nullptr, ldbar, h, grp, n0);
+        if ((int)blockIdx.x < nitems) issue_dt(blockIdx.x, 0);
     }
-    if (geo.use) ++ld_issued;
-    load_chunk_meta(a, b, h, n0, len, L, sgoff, sdt);
+    if ((int)blockIdx.x < nitems) ++dt_issued;
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -329,6 +346,34 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncthreads();
         return *abort_flag == 0;
     };
+    // persistent: this CTA takes items blockIdx.x, + gridDim.x, ...
+    for (int item = blockIdx.x, li = 0; item < nitems; item += gridDim.x, ++li) {
+    h = item % a.nh;
+    c = (item / a.nh) % a.nchunks;
+    b = item / (a.nh * a.nchunks) + geo.zbase;
+    n0 = c * L;
+    len = min(L, a.N - n0);
+    grp = h / (a.nh / a.G);
+    Ah = a.A[h];
+    Dh2 = 2.f * a.D[h];
+    float *sdt = sdt_buf + (li & 1) * kMaxChunk;
+    if (tid == 0 && geo.use) {
+        // TMA boxes need no grid offsets: sub-chunk 0's rows are requested first
+        tma_rows(&mx, &mB, &mC, geo, sX, sB, nullptr, ldbar, h, grp, n0);
+        // the output phase reads x and B again (from L2, read in phase 1) and C for
+        // the first time: C of every sub-chunk into L2 now
+        for (int k = 0; k < nsub; ++k) {
+            const int sp = n0 + k * kSub, a0 = sp % geo.n0, q = sp / geo.n0;
+            tc::tma_prefetch_5d(&mC, 0, grp, a0, q % geo.n1, q / geo.n1);
+        }
+    }
+    if (geo.use) ++ld_issued;
+    else chunk_offsets(a, n0, len, L, sgoff);  // the gathers need the grid offsets
+    // this item's dt (requested during the previous item, or at the start)
+    if (!tc::mbar_wait(dtbar, dt_phase & 1u, a.err)) *abort_flag = 1;
+    ++dt_phase;
+    __syncthreads();
+    if (*abort_flag) goto cleanup;
     // x, B of sub-chunk 0 are in flight while the decay factors are prepared
     if (!geo.use) issue_rows(sX, sB, nullptr, 0);  // (the TMA batch is already in flight)
     sub_cumsums(sdt, scum, Ah, nsub, false, sred);
@@ -470,6 +515,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
     };
     write_h(0);
+    if (item + (int)gridDim.x < nitems) {
+        // the next item's dt into the other buffer (last read by the item before this
+        // one), and its first rows into L2
+        if (tid == 0) {
+            const int nx = item + gridDim.x;
+            issue_dt(nx, (li + 1) & 1);
+            if (geo.use) {
+                const int nh_ = nx % a.nh, nc = (nx / a.nh) % a.nchunks, sp = nc * L;
+                const int a0 = sp % geo.n0, q = sp / geo.n0;
+                tc::tma_prefetch_5d(&mx, 0, nh_, a0, q % geo.n1, q / geo.n1);
+                tc::tma_prefetch_5d(&mB, 0, nh_ / (a.nh / a.G), a0, q % geo.n1, q / geo.n1);
+            }
+        }
+        ++dt_issued;
+    }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     if (!rows_wait()) goto cleanup;
@@ -621,18 +681,14 @@ __global__ void __launch_bounds__(kThreads, 2)
             issue_rows(sX, sB, sC, k + 1);
         }
 
-        // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r. Each warp stages its
-        // 32 half rows (64 bytes) in its own 2 KB of the free M tiles, then stores them
-        // at the grid positions of their tokens, eight half rows per store instruction.
+        // epilogue: columns 32g .. 32g+31 of y_r = Acc_r + 2 D x_r, rounded to bf16
         {
-            uint8_t *stg = sM + warp * 2048;
             uint32_t acc2[2][16];
             tc::tmem_ld16(tc::tmem_addr(tAcc, lane_base, 32 * g), acc2[0]);
             tc::tmem_ld16(tc::tmem_addr(tAcc, lane_base, 32 * g + 16), acc2[1]);
             tc::tmem_wait_ld();
-            const int lr = r & 31;  // this thread's row within the warp
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            // 16-byte chunk q of this thread's half row (eight bf16 values)
+            auto chunk16 = [&](int q) {
                 const uint32_t *acc = acc2[q >> 1] + 8 * (q & 1);
                 const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
                 uint32_t o4[4];
@@ -643,19 +699,46 @@ __global__ void __launch_bounds__(kThreads, 2)
                                                                 __uint_as_float(acc[2 * e + 1])));
                     o4[e] = bf2(y2.x, y2.y);
                 }
-                *reinterpret_cast<uint4 *>(stg + lr * 64 + ((q ^ ((lr >> 1) & 3)) << 4)) =
-                    make_uint4(o4[0], o4[1], o4[2], o4[3]);
-            }
-            __syncwarp();
-            const int row0 = r & ~31;
+                return make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            };
+            if (geo.use) {
+                // the sub-chunk's rows form one box of the grid: stage them in the 128-byte
+                // swizzle (one of the two free M tiles, alternating) and store the box by TMA;
+                // rows past the sequence end fall outside the tensor and are not written
+                uint8_t *stg = sM + (k & 1) * kTile;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int rr = i * 8 + (lane >> 2), q = lane & 3, nn = k * kSub + row0 + rr;
-                if (nn < len) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(stg + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4));
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
-                                         (((size_t)b * a.N + sgoff[nn]) * a.nh + h) * 64 + 32 * g + q * 8;
-                    *reinterpret_cast<uint4 *>(dst) = v;
+                for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4 *>(stg + tc::sw128(r, 4 * g + q)) = chunk16(q);
+                tc::fence_proxy_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    const int sp = n0 + k * kSub, a0 = sp % geo.n0, qq = sp / geo.n0;
+                    tc::tma_store_5d(&mO, stg, 0, h, a0, qq % geo.n1, qq / geo.n1);
+                    tc::bulk_commit();
+                    // the store before this one has read its tile, which the next
+                    // sub-chunk's epilogue writes (after the barriers in between)
+                    tc::bulk_wait_read<1>();
+                }
+            } else {
+                // each warp stages its 32 half rows (64 bytes) in its own 2 KB of the free M
+                // tiles, then stores them at the grid positions of their tokens, eight half
+                // rows per store instruction
+                uint8_t *stg = sM + warp * 2048;
+                const int lr = r & 31;  // this thread's row within the warp
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(stg + lr * 64 + ((q ^ ((lr >> 1) & 3)) << 4)) = chunk16(q);
+                __syncwarp();
+                const int row0 = r & ~31;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int rr = i * 8 + (lane >> 2), q = lane & 3, nn = k * kSub + row0 + rr;
+                    if (nn < len) {
+                        const uint4 v =
+                            *reinterpret_cast<const uint4 *>(stg + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4));
+                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
+                                             (((size_t)b * a.N + sgoff[nn]) * a.nh + h) * 64 + 32 * g + q * 8;
+                        *reinterpret_cast<uint4 *>(dst) = v;
+                    }
                 }
             }
         }
@@ -665,11 +748,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::tc_fence_after();
     }
     }
+    // the next item's phase 1 writes the M tiles, which the last output stores read
+    if (tid == 0) tc::bulk_wait_read<0>();
+    // this item's dt buffer is written next by a bulk load (async proxy)
+    tc::fence_proxy_async_smem();
+    __syncthreads();
+    }
 
 cleanup:
     tc::cp_async_wait_all();
-    // after a timeout a TMA batch may still be landing: a second bounded wait for it
+    // after a timeout a TMA batch or a dt load may still be landing: bounded waits for them
     if (ld_issued > ld_phase && tid == 0) tc::mbar_wait(ldbar, ld_phase & 1u, nullptr);
+    if (dt_issued > dt_phase && tid == 0) tc::mbar_wait(dtbar, dt_phase & 1u, nullptr);
+    if (tid == 0) tc::bulk_wait_all();  // output stores read shared memory until they complete
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -799,6 +890,11 @@ __global__ void __launch_bounds__(kThreads, 4)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // chunk_out loads this chunk's dt in scan order with one bulk copy
+    {
+        float4 *dst = reinterpret_cast<float4 *>(a.dt_scan + (((size_t)b * a.nh + h) * a.nchunks + c) * L);
+        for (int i = tid; i < L / 4; i += kThreads) dst[i] = reinterpret_cast<const float4 *>(sdt)[i];
+    }
     sub_cumsums(sdt, scum, Ah, nsub, true, sred);
     const float cend = scum[L - 1];
 
@@ -1020,7 +1116,7 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
     const int nsub = a.Q / kSub;
     // TMA row boxes when the scan order allows them: one launch per batch element
     struct Maps {
-        CUtensorMap x, b, c;
+        CUtensorMap x, b, c, o;
     };
     const ScanBox sb = scan_box(a.mode, a.T, a.H, a.W);
     auto build_maps = [&](int bb, Maps &m) {
@@ -1033,7 +1129,8 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
         const size_t tok = (size_t)bb * a.N;
         return tmap_bf16_5d(&m.x, static_cast<const __nv_bfloat16 *>(a.x) + tok * a.nh * 64, dx, sx, box) &&
                tmap_bf16_5d(&m.b, static_cast<const __nv_bfloat16 *>(a.B) + tok * a.G * 64, db, sbs, box) &&
-               tmap_bf16_5d(&m.c, static_cast<const __nv_bfloat16 *>(a.C) + tok * a.G * 64, db, sbs, box);
+               tmap_bf16_5d(&m.c, static_cast<const __nv_bfloat16 *>(a.C) + tok * a.G * 64, db, sbs, box) &&
+               tmap_bf16_5d(&m.o, static_cast<const __nv_bfloat16 *>(a.out) + tok * a.nh * 64, dx, sx, box);
     };
     Maps maps = {};
     TmaRows geo = {0, 1, 1, 0};
@@ -1059,12 +1156,17 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
         Phase ph(MATE_PHASE_STATE_PASS, s);
         ssd_state_chain_kernel<<<dim3(4096 / 8 / 256, a.nh * a.batch, 2), 256, 0, s>>>(a);
     }
+    // chunk_out is persistent: two CTAs per SM walk the (head, chunk, batch) items
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nitems = a.nh * a.nchunks * zdim;
+    const int grid = std::min(nitems, 2 * std::max(nsm, 1));
     for (int l = 0; l < launches; ++l) {
         if (geo.use && !build_maps(l, maps)) return cudaErrorInvalidValue;
         geo.zbase = geo.use ? l : 0;
         Phase ph(MATE_PHASE_CHUNK_OUT, s);
-        ssd_chunk_out_tc_kernel<<<dim3(a.nh, a.nchunks, zdim), kThreads, kSmemBytes, s>>>(a, nsub, maps.x, maps.b,
-                                                                                         maps.c, geo);
+        ssd_chunk_out_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a, nsub, maps.x, maps.b, maps.c, maps.o, geo,
+                                                                  nitems);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

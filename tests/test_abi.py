@@ -145,13 +145,18 @@ def test_dispatch_by_storage_type():
 
 
 def test_workspace_layout_by_storage_type():
-    """Chunk states take 2 bytes per element for bf16 storage and 4 for fp32."""
-    def expected(nchunks, nh, state_bytes):
+    """Chunk states take 2 bytes per element for bf16 storage and 4 for fp32;
+    bf16 storage adds dt in scan order (fp32, padded to whole chunks)."""
+    def expected(nchunks, nh, state_bytes, chunk):
         align = lambda v: (v + 255) // 256 * 256
         states = align(nchunks * nh * 64 * 64 * state_bytes)
-        return 2 * states + align(nchunks * nh * 4)
+        dt_scan = align(nchunks * chunk * nh * 4) if state_bytes == 2 else 0
+        return 2 * states + align(nchunks * nh * 4) + dt_scan
     # 2,048 tokens, chunk 256 -> 8 chunks, 4 heads of 64 x 64, no review tokens
     assert api.mate_bissd_workspace_bytes(8, 16, 16, None, _dims(nheads=4, headdim=64, dstate=64, chunk=256,
-                                                                 dtype=1)) == expected(8, 4, 2)
+                                                                 dtype=1)) == expected(8, 4, 2, 256)
     assert api.mate_bissd_workspace_bytes(8, 16, 16, None, _dims(nheads=4, headdim=64, dstate=64, chunk=256,
-                                                                 dtype=0)) == expected(8, 4, 4)
+                                                                 dtype=0)) == expected(8, 4, 4, 256)
+    # 1,200 tokens, chunk 512 -> 3 chunks (the last one partial): dt padded to 1,536 positions
+    assert api.mate_bissd_workspace_bytes(5, 12, 20, None, _dims(nheads=4, headdim=64, dstate=64, chunk=512,
+                                                                 dtype=1)) == expected(3, 4, 2, 512)
