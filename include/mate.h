@@ -227,6 +227,17 @@ int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, i
 int mate_debug_rms_map(int T, int H, int W, int scan_mode, int flip, int32_t *out_dev, void *stream);
 
 /*
+ * Test hook for the integer division the tensor-core SSD kernels use for the
+ * scan-order index map and the review cells (a divisor fixed per call,
+ * multiply-high form; no counterpart in the pages): q[i] = n[i] / d for
+ * count values, computed on the host with the same code the kernels run.
+ * n and q are host arrays (caller-owned); every n[i] must be below 2^31 and
+ * 1 <= d < 2^31. Returns MATE_OK, or MATE_ERR_INVALID_ARG (nothing written)
+ * for null arrays or values out of range.
+ */
+int mate_debug_fastdiv(const uint32_t *n, uint32_t *q, size_t count, uint32_t d);
+
+/*
  * Debug export of the TESA window partition the kernels use: out_win_dev[g]
  * = window id of grid token g, windows numbered in (t, h, w) order of their
  * first token. out_win_dev holds T*H*W int32 (device memory, caller-owned).

@@ -30,6 +30,7 @@ EXPORTS = (
     "tesa_fwd",
     "mate_debug_rms_map",
     "mate_debug_tesa_map",
+    "mate_debug_fastdiv",
     "mate_last_error",
     "mate_status_string",
     "mate_version",
@@ -89,6 +90,8 @@ def load() -> ctypes.CDLL:
     L.mate_last_error.restype = ctypes.c_int
     L.mate_status_string.argtypes = [ctypes.c_int]
     L.mate_status_string.restype = ctypes.c_char_p
+    L.mate_debug_fastdiv.argtypes = [_vp, _vp, ctypes.c_size_t, ctypes.c_uint32]
+    L.mate_debug_fastdiv.restype = ctypes.c_int
     L.mate_version.argtypes = []
     L.mate_version.restype = ctypes.c_int
     L.mate_set_phase_hook.argtypes = [PHASE_HOOK, ctypes.c_void_p]

@@ -8,6 +8,37 @@
 
 namespace mate {
 
+// Division of non-negative 32-bit integers below 2^31 by a divisor fixed at
+// launch (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", PLDI 1994, figure 4.1): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (mulhi(m, n) + n) >> l. Three
+// integer instructions instead of a general division.
+struct FastDiv {
+    uint32_t d, m, l;
+};
+
+inline FastDiv make_fastdiv(uint32_t d)
+{
+    FastDiv f;
+    f.d = d;
+    f.l = 0;
+    while (f.l < 31 && (1u << f.l) < d) ++f.l;
+    f.m = (uint32_t)((((uint64_t)1 << 32) * (((uint64_t)1 << f.l) - d)) / d + 1);
+    return f;
+}
+
+#ifdef __CUDACC__
+__host__ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f)
+{
+#ifdef __CUDA_ARCH__
+    const uint32_t hi = __umulhi(n, f.m);
+#else
+    const uint32_t hi = (uint32_t)(((uint64_t)n * f.m) >> 32);
+#endif
+    return (hi + n) >> f.l;
+}
+#endif
+
 // Everything one bi-SSD call needs, resolved on the host.
 struct SsdArgs {
     const void *x;
@@ -27,6 +58,8 @@ struct SsdArgs {
     int Tp, Hp, Wp, Np;      // pooled grid and its token count
     int pool_splits;         // each pooling box is summed in this many parts
     int bf16;                // 1: x, B, C, out are bf16; 0: fp32
+    // the same divisors for the RMS index map and the review cells, as FastDiv
+    FastDiv dT, dH, dW, dHW, dpt, dph, dpw;
     // workspace carve-outs (fp32)
     float *states_f;         // (batch, nh, nchunks, P, Ns): chunk-local forward states,
                              //   overwritten by the state entering each chunk (the

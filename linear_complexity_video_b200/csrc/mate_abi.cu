@@ -100,6 +100,11 @@ int ssd_shape(int T, int H, int W, const int *pool, const mate_ssd_dims *d, int 
     a.mode = scan_mode;
     a.dirs = dirs;
     a.bf16 = d->dtype == MATE_BF16;
+    a.dT = make_fastdiv(T);
+    a.dH = make_fastdiv(H);
+    a.dW = make_fastdiv(W);
+    a.dHW = make_fastdiv((uint32_t)(H * W));
+    a.dpt = a.dph = a.dpw = make_fastdiv(1);
     const bool review = pool && (pool[0] || pool[1] || pool[2]);
     if (review) {
         if (pool[0] <= 0 || pool[1] <= 0 || pool[2] <= 0) return MATE_ERR_INVALID_ARG;
@@ -112,6 +117,9 @@ int ssd_shape(int T, int H, int W, const int *pool, const mate_ssd_dims *d, int 
         a.Hp = H / pool[1];
         a.Wp = W / pool[2];
         a.Np = a.Tp * a.Hp * a.Wp;
+        a.dpt = make_fastdiv(a.pt);
+        a.dph = make_fastdiv(a.ph);
+        a.dpw = make_fastdiv(a.pw);
         // split each pooling box so that the pooling grid covers the GPU a few times over
         const int64_t box = (int64_t)a.pt * a.ph * a.pw;
         const int64_t blocks = (int64_t)a.Np * a.batch * ((a.nh * a.P + a.nh + a.G * a.Ns) / 8 / 256 + 1);
@@ -295,6 +303,17 @@ int mate_debug_rms_map(int T, int H, int W, int scan_mode, int flip, int32_t *ou
     if ((int64_t)T * H * W >= ((int64_t)1 << 31)) return MATE_ERR_INVALID_ARG;
     cudaError_t err = launch_rms_map(T, H, W, scan_mode, flip, out_dev, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
+int mate_debug_fastdiv(const uint32_t *n, uint32_t *q, size_t count, uint32_t d)
+{
+    if ((!n || !q) && count) return MATE_ERR_INVALID_ARG;
+    if (d < 1 || d >= (1u << 31)) return MATE_ERR_INVALID_ARG;
+    for (size_t i = 0; i < count; ++i)
+        if (n[i] >= (1u << 31)) return MATE_ERR_INVALID_ARG;
+    const FastDiv f = make_fastdiv(d);
+    for (size_t i = 0; i < count; ++i) q[i] = fdiv(n[i], f);
+    return MATE_OK;
 }
 
 int mate_debug_tesa_map(int T, int H, int W, int Tw, int Sw, const int shift[3], int32_t *out_win_dev, void *stream)

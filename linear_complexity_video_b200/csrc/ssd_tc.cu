@@ -123,6 +123,32 @@ __device__ __forceinline__ void wait_loads(bool newer_pending)
         asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
+// rms_grid_offset with the divisions by T, H, W and H*W taken by the launch-time
+// FastDiv divisors (scan positions and grid offsets are below 2^31).
+__device__ __forceinline__ int rms_offset_fast(int n, const SsdArgs &a)
+{
+    const uint32_t u = (uint32_t)n;
+    switch (a.mode) {
+    case MATE_SCAN_SR:
+        return n;
+    case MATE_SCAN_SC: {
+        const uint32_t t = fdiv(u, a.dHW), rem = u - t * a.dHW.d;
+        const uint32_t w = fdiv(rem, a.dH), hh = rem - w * a.dH.d;
+        return (int)(t * a.dHW.d + hh * a.dW.d + w);
+    }
+    case MATE_SCAN_TR: {
+        const uint32_t sp = fdiv(u, a.dT), t = u - sp * a.dT.d;
+        const uint32_t hh = fdiv(sp, a.dW), w = sp - hh * a.dW.d;
+        return (int)((t * a.dH.d + hh) * a.dW.d + w);
+    }
+    default: {  // MATE_SCAN_TC
+        const uint32_t sp = fdiv(u, a.dT), t = u - sp * a.dT.d;
+        const uint32_t w = fdiv(sp, a.dH), hh = sp - w * a.dH.d;
+        return (int)((t * a.dH.d + hh) * a.dW.d + w);
+    }
+    }
+}
+
 // Per-chunk setup shared by chunk_state and chunk_out: grid offsets and dt of
 // the chunk's L positions (zero past the sequence end).
 __device__ __forceinline__ void load_chunk_meta(const SsdArgs &a, int b, int h, int n0, int len, int L, int *goff,
@@ -132,7 +158,7 @@ __device__ __forceinline__ void load_chunk_meta(const SsdArgs &a, int b, int h, 
         float d = 0.f;
         int g = 0;
         if (n < len) {
-            g = rms_grid_offset(n0 + n, a.T, a.H, a.W, a.mode);
+            g = rms_offset_fast(n0 + n, a);
             d = a.dt[((size_t)b * a.N + g) * a.nh + h];
         }
         goff[n] = g;
@@ -143,7 +169,7 @@ __device__ __forceinline__ void load_chunk_meta(const SsdArgs &a, int b, int h, 
 // Grid offsets of the chunk's L positions (0 past the sequence end).
 __device__ __forceinline__ void chunk_offsets(const SsdArgs &a, int n0, int len, int L, int *goff)
 {
-    for (int n = threadIdx.x; n < L; n += kThreads) goff[n] = n < len ? rms_grid_offset(n0 + n, a.T, a.H, a.W, a.mode) : 0;
+    for (int n = threadIdx.x; n < L; n += kThreads) goff[n] = n < len ? rms_offset_fast(n0 + n, a) : 0;
 }
 
 // Inclusive cumulative sums of A*dt within each 128-token sub-chunk (warp w
@@ -921,9 +947,10 @@ __global__ void __launch_bounds__(kThreads, 4)
                 const int n0r = k * kSub + rbase + RUN * lane_run(j);
                 int cell = -1;
                 if (n0r < len) {
-                    const int gg = sgoff[n0r], hw = a.H * a.W;
-                    const int t = gg / hw, hh = (gg - t * hw) / a.W, ww = gg - t * hw - hh * a.W;
-                    cell = b * a.Np + ((t / a.pt) * a.Hp + hh / a.ph) * a.Wp + ww / a.pw;
+                    const uint32_t gg = (uint32_t)sgoff[n0r];
+                    const uint32_t t = fdiv(gg, a.dHW), rem = gg - t * a.dHW.d;
+                    const uint32_t hh = fdiv(rem, a.dW), ww = rem - hh * a.dW.d;
+                    cell = b * a.Np + (int)((fdiv(t, a.dpt) * a.Hp + fdiv(hh, a.dph)) * a.Wp + fdiv(ww, a.dpw));
                 }
                 if (cell != runs.cell[j]) {
                     run_flush<RUN>(a, runs, j, h, grp, c4, with_d, with_b);

@@ -160,3 +160,42 @@ def test_workspace_layout_by_storage_type():
     # 1,200 tokens, chunk 512 -> 3 chunks (the last one partial): dt padded to 1,536 positions
     assert api.mate_bissd_workspace_bytes(5, 12, 20, None, _dims(nheads=4, headdim=64, dstate=64, chunk=512,
                                                                  dtype=1)) == expected(3, 4, 2, 512)
+
+
+def test_fastdiv_matches_integer_division():
+    """The kernels' multiply-high division (Granlund and Montgomery 1994,
+    figure 4.1) against exact integer division: every divisor the index maps
+    can meet on small grids, powers of two and their neighbours, large odd
+    divisors, and dividends at the ends of the range."""
+    import numpy as np
+
+    L = mate.load()
+    rng = np.random.default_rng(0)
+    top = (1 << 31) - 1
+    divisors = list(range(1, 300)) + [(1 << k) + e for k in range(1, 31) for e in (-1, 0, 1)] + \
+        [top, top - 1, 1_000_003, 73_728, 147_456, 2_359_296]
+    for d in divisors:
+        if not 1 <= d <= top:
+            continue
+        n = np.concatenate([np.arange(0, 2048, dtype=np.uint64),
+                            rng.integers(0, 1 << 31, 4096, dtype=np.uint64),
+                            np.array([top, top - 1, d, d - 1, d + 1, 2 * d - 1, top // d * d, top // d * d - 1],
+                                     dtype=np.uint64)])
+        n = n[n <= top].astype(np.uint32)
+        q = np.empty_like(n)
+        assert L.mate_debug_fastdiv(n.ctypes.data, q.ctypes.data, n.size, d) == _lib.MATE_OK
+        assert np.array_equal(q, n // np.uint32(d)), d
+
+
+def test_fastdiv_rejects_out_of_range():
+    import numpy as np
+
+    L = mate.load()
+    n = np.array([1 << 31], dtype=np.uint32)
+    q = np.zeros(1, dtype=np.uint32)
+    assert L.mate_debug_fastdiv(n.ctypes.data, q.ctypes.data, 1, 3) == _lib.MATE_ERR_INVALID_ARG
+    n[0] = 5
+    assert L.mate_debug_fastdiv(n.ctypes.data, q.ctypes.data, 1, 0) == _lib.MATE_ERR_INVALID_ARG
+    assert L.mate_debug_fastdiv(n.ctypes.data, q.ctypes.data, 1, 1 << 31) == _lib.MATE_ERR_INVALID_ARG
+    assert L.mate_debug_fastdiv(None, None, 1, 3) == _lib.MATE_ERR_INVALID_ARG
+    assert q[0] == 0
