@@ -442,8 +442,9 @@ def time_config(cfg, mode, steps, warmup, seed=0):
 
 
 def run_report(args):
-    """Every bf16 grid in every scan order it lists, then the N sweep with a
-    linearity fit. One JSON line per measurement, then a summary line."""
+    """Every bf16 grid in every scan order it lists, the headline grid in the
+    zigzag comparison order, then the N sweep with a linearity fit. One JSON
+    line per measurement, then a summary line."""
     import numpy as np
     import torch
 
@@ -461,6 +462,15 @@ def run_report(args):
                               "mtokens_per_s": round(cfg.tokens / ms / 1e3, 3),
                               "path_hbm_frac": round(path_bytes / (ms / 1e3) / 1e9 / hbm, 4),
                               "phase_ms": phases}), flush=True)
+    # the pages' scan ablation (paper review 5.5 Table 2: Zigzag instead of RMS) at kernel
+    # level: the headline grid in its RMS order and in the zigzag comparison order
+    cfg = workloads.CONFIGS[workloads.HEADLINE]
+    ms_rms, ph_rms = time_config(cfg, cfg.modes[0], args.steps, args.warmup)
+    ms_zz, ph_zz = time_config(cfg, workloads.ZZ, args.steps, args.warmup)
+    print(json.dumps({"report": "scan_ablation", "workload": cfg.name, "tokens": cfg.tokens,
+                      "rms_scan": workloads.MODE_NAMES[cfg.modes[0]], "rms_ms_per_step": round(ms_rms, 4),
+                      "zigzag_ms_per_step": round(ms_zz, 4), "zigzag_over_rms": round(ms_zz / ms_rms, 4),
+                      "rms_phase_ms": ph_rms, "zigzag_phase_ms": ph_zz}), flush=True)
     Ns, ts = [], []
     for cfg in workloads.sweep_configs():
         ms, phases = time_config(cfg, cfg.modes[0], args.steps, args.warmup)

@@ -75,6 +75,17 @@ extern "C" {
 #define MATE_SCAN_SC 1
 #define MATE_SCAN_TR 2
 #define MATE_SCAN_TC 3
+/* Zigzag scan, the alternative the pages compare RMS against (QbitAI article,
+ * method section; paper review, 5.5 Table 2: "Zigzag ... 144 s"). The pages
+ * do not define it; it is read here as the 3D boustrophedon in which every
+ * step moves to a neighbouring token: frames in time order, the rows of even
+ * frames top to bottom and of odd frames bottom to top, and global row
+ * R = t*H + i (i = row counted in visiting order) walked along W left to
+ * right when R is even, right to left when R is odd:
+ *   n = (t*H + i)*W + j,  h = t even ? i : H-1-i,  w = R even ? j : W-1-j.
+ * Its sub-chunks are not boxes of the grid, so the kernels gather its rows.
+ * The flipped scan is defined as for the RMS orders. */
+#define MATE_SCAN_ZZ 4
 
 /* directions of the bidirectional scan (test and diagnosis aid) */
 #define MATE_DIR_FWD 1 /* the scan in RMS order only          */
@@ -117,7 +128,8 @@ size_t mate_bissd_workspace_bytes(int T, int H, int W, const int review_pool[3],
  * order with optional review tokens (paper review, MA-Branch items 1-3).
  *
  * For each batch element and head h, let X be the grid unrolled in scan
- * order `scan_mode` (N = T*H*W tokens). With state s (headdim x dstate,
+ * order `scan_mode` (MATE_SCAN_SR .. MATE_SCAN_TC, or MATE_SCAN_ZZ for the
+ * zigzag comparison; N = T*H*W tokens). With state s (headdim x dstate,
  * zero at the start of every scanned sequence) the scan computes
  *     s_n = exp(dt_n * A[h]) * s_{n-1} + dt_n * x_n B_n^T
  *     y_n = s_n C_n + D[h] * x_n

@@ -32,6 +32,14 @@ __host__ __device__ __forceinline__ int rms_grid_offset(int n, int T, int H, int
         const int h = s / W, w = s - h * W;
         return (t * H + h) * W + w;
     }
+    case MATE_SCAN_ZZ: {  // 3D boustrophedon (mate.h)
+        const int hw = H * W;
+        const int t = n / hw, r = n - t * hw;
+        const int i = r / W, j = r - i * W;
+        const int h = (t & 1) ? H - 1 - i : i;
+        const int w = ((t * H + i) & 1) ? W - 1 - j : j;
+        return (t * H + h) * W + w;
+    }
     default: {  // MATE_SCAN_TC
         const int s = n / T, t = n - s * T;
         const int w = s / H, h = s - w * H;

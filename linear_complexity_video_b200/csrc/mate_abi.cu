@@ -79,7 +79,7 @@ int ssd_shape(int T, int H, int W, const int *pool, const mate_ssd_dims *d, int 
     const int64_t N = (int64_t)T * H * W;
     if (N >= ((int64_t)1 << 31) || N * d->batch >= ((int64_t)1 << 40)) return MATE_ERR_INVALID_ARG;
     if (d->nheads % d->ngroups) return MATE_ERR_INVALID_ARG;
-    if (scan_mode < 0 || scan_mode > 3) return MATE_ERR_INVALID_ARG;
+    if (scan_mode < 0 || scan_mode > MATE_SCAN_ZZ) return MATE_ERR_INVALID_ARG;
     const int dirs = d->directions == 0 ? MATE_DIR_BI : d->directions;
     if (dirs < 1 || dirs > 3) return MATE_ERR_INVALID_ARG;
     if (d->dtype != MATE_F32 && d->dtype != MATE_BF16) return MATE_ERR_UNSUPPORTED;
@@ -299,7 +299,8 @@ int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, i
 
 int mate_debug_rms_map(int T, int H, int W, int scan_mode, int flip, int32_t *out_dev, void *stream)
 {
-    if (T <= 0 || H <= 0 || W <= 0 || scan_mode < 0 || scan_mode > 3 || !out_dev) return MATE_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || W <= 0 || scan_mode < 0 || scan_mode > MATE_SCAN_ZZ || !out_dev)
+        return MATE_ERR_INVALID_ARG;
     if ((int64_t)T * H * W >= ((int64_t)1 << 31)) return MATE_ERR_INVALID_ARG;
     cudaError_t err = launch_rms_map(T, H, W, scan_mode, flip, out_dev, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;

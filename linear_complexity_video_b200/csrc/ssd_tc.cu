@@ -141,6 +141,13 @@ __device__ __forceinline__ int rms_offset_fast(int n, const SsdArgs &a)
         const uint32_t hh = fdiv(sp, a.dW), w = sp - hh * a.dW.d;
         return (int)((t * a.dH.d + hh) * a.dW.d + w);
     }
+    case MATE_SCAN_ZZ: {  // 3D boustrophedon (mate.h)
+        const uint32_t t = fdiv(u, a.dHW), rem = u - t * a.dHW.d;
+        const uint32_t i = fdiv(rem, a.dW), j = rem - i * a.dW.d;
+        const uint32_t hh = (t & 1) ? a.dH.d - 1 - i : i;
+        const uint32_t w = ((t * a.dH.d + i) & 1) ? a.dW.d - 1 - j : j;
+        return (int)((t * a.dH.d + hh) * a.dW.d + w);
+    }
     default: {  // MATE_SCAN_TC
         const uint32_t sp = fdiv(u, a.dT), t = u - sp * a.dT.d;
         const uint32_t w = fdiv(sp, a.dH), hh = sp - w * a.dH.d;
@@ -1121,7 +1128,9 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
     // long along the scan's fastest axis and the channel blocks allow 16-byte atomics
     int run = 0;
     if (a.review) {
-        const int r0 = a.mode == MATE_SCAN_SR ? a.pw : (a.mode == MATE_SCAN_SC ? a.ph : a.pt);
+        // (the zigzag scan walks W inside each row, either way: runs of pw along W)
+        const int r0 = (a.mode == MATE_SCAN_SR || a.mode == MATE_SCAN_ZZ) ? a.pw
+                       : (a.mode == MATE_SCAN_SC ? a.ph : a.pt);
         if ((r0 == 4 || r0 == 8) && a.nh % 4 == 0 && (a.G * a.Ns) % 4 == 0) run = r0;
     }
     auto st_kernel = run == 8 ? ssd_chunk_state_tc_kernel<8>

@@ -64,6 +64,8 @@ ScanBox scan_box(int mode, int T, int H, int W)
     case MATE_SCAN_TR:  // (h, w, t): t fastest
         n[0] = T; s[0] = st; n[1] = W; s[1] = sw; n[2] = H; s[2] = sh;
         break;
+    case MATE_SCAN_ZZ:  // rows alternate direction: no sub-chunk is a box of the grid
+        return sb;
     default:            // MATE_SCAN_TC (w, h, t): t fastest
         n[0] = T; s[0] = st; n[1] = H; s[1] = sh; n[2] = W; s[2] = sw;
         break;

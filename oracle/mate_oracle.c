@@ -37,6 +37,8 @@
  *      congruent to the shift modulo the window size; the windows at the two
  *      ends are partial. Plain softmax(q k^T / sqrt(d)) v per head inside each
  *      window, no mask inside a window, no position bias.
+ *   R6 Zigzag scan (named, not defined, by the pages): the 3D boustrophedon
+ *      of oracle_zigzag, used only as the comparison order.
  */
 #include <math.h>
 #include <stdint.h>
@@ -82,12 +84,36 @@ int oracle_unroll(int T, int H, int W, const int priority[3], int32_t *seq)
     return ORACLE_OK;
 }
 
-/* The scan sequence of a mode, optionally flipped ([Review] MA-Branch item 2:
- * every layer scans the sequence and its flip; reading R2). */
+/* The Zigzag scan the pages set against RMS ([QbitAI] method section: Zigzag
+ * and Hilbert scans keep neighbours together but need costly reorderings;
+ * [Review] 5.5 Table 2, "Zigzag"). The pages do not define it; reading R6:
+ * a 3D boustrophedon whose every step moves to a neighbouring token. Frames
+ * are visited in time order; even frames take their rows top to bottom, odd
+ * frames bottom to top; the k-th row visited overall (k from 0) is walked
+ * along W left to right when k is even and right to left when k is odd. */
+int oracle_zigzag(int T, int H, int W, int32_t *seq)
+{
+    if (T <= 0 || H <= 0 || W <= 0 || !seq) return ORACLE_EINVAL;
+    int64_t n = 0, row = 0;
+    for (int t = 0; t < T; ++t) {
+        for (int i = 0; i < H; ++i, ++row) {
+            const int h = (t % 2 == 0) ? i : H - 1 - i;
+            for (int j = 0; j < W; ++j) {
+                const int w = (row % 2 == 0) ? j : W - 1 - j;
+                seq[n++] = (int32_t)(((int64_t)t * H + h) * W + w);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* The scan sequence of a mode (0-3: the RMS orders, 4: Zigzag), optionally
+ * flipped ([Review] MA-Branch item 2: every layer scans the sequence and its
+ * flip; reading R2). */
 int oracle_rms_sequence(int T, int H, int W, int mode, int flip, int32_t *seq)
 {
-    if (mode < 0 || mode > 3) return ORACLE_EINVAL;
-    int rc = oracle_unroll(T, H, W, kScanPriority[mode], seq);
+    if (mode < 0 || mode > 4) return ORACLE_EINVAL;
+    int rc = mode == 4 ? oracle_zigzag(T, H, W, seq) : oracle_unroll(T, H, W, kScanPriority[mode], seq);
     if (rc != ORACLE_OK || !flip) return rc;
     int64_t N = (int64_t)T * H * W;
     for (int64_t i = 0, j = N - 1; i < j; ++i, --j) {
@@ -206,7 +232,7 @@ int oracle_bissd(int batch, int T, int H, int W, int nh, int P, int Ns, int G,
                  int mode, const int *pool, double *out)
 {
     if (batch <= 0 || T <= 0 || H <= 0 || W <= 0 || nh <= 0 || P <= 0 || Ns <= 0 || G <= 0 ||
-        nh % G || mode < 0 || mode > 3)
+        nh % G || mode < 0 || mode > 4)
         return ORACLE_EINVAL;
     const int review = pool && (pool[0] || pool[1] || pool[2]);
     if (review && (pool[0] <= 0 || pool[1] <= 0 || pool[2] <= 0 ||

@@ -342,6 +342,32 @@ def pin_tesa_special(o):
     _close(got[0], want, 1e-13, "q = 0 gives the window mean")
 
 
-ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_pool, pin_scan_dual,
+def pin_zigzag(o):
+    """The zigzag comparison order (mode 4). The pages name the Zigzag scan
+    (QbitAI method section; paper review 5.5 Table 2) without defining it; the
+    reading is the 3D boustrophedon. These properties fix that order
+    uniquely: a bijection that starts at grid token 0 and first moves along
+    +W; frames visited whole and in time order, each row (t, h) visited
+    whole along W; every step to a neighbouring token (one unit in one
+    axis). The flip is the reversal, as for the RMS orders."""
+    for (T, H, W) in [(2, 2, 3), (3, 4, 5), (1, 5, 1), (4, 1, 6), (3, 3, 2), (2, 7, 4)]:
+        N = T * H * W
+        seq = o.rms_sequence(T, H, W, 4)
+        assert np.array_equal(np.sort(seq), np.arange(N)), "not a bijection"
+        t, h, w = seq // (H * W), (seq // W) % H, seq % W
+        assert seq[0] == 0 and (N == 1 or W == 1 or seq[1] == 1), "does not start at token 0 along +W"
+        assert np.all(t == np.repeat(np.arange(T), H * W)), "frames not whole and in time order"
+        rows = (t * H + h).reshape(T * H, W)
+        assert np.all(rows == rows[:, :1]), "a row is not visited whole along W"
+        if N > 1:
+            step = np.abs(np.diff(t)) + np.abs(np.diff(h)) + np.abs(np.diff(w))
+            assert np.all(step == 1), "a step does not move to a neighbouring token"
+        assert np.array_equal(o.rms_sequence(T, H, W, 4, flip=True), seq[::-1]), "flip is not n -> N-1-n"
+    # 2 x 2 x 3 written out by hand: frame 0 rows h = 0 (w ->), h = 1 (w <-);
+    # frame 1 rows h = 1 (w ->), h = 0 (w <-)
+    assert o.rms_sequence(2, 2, 3, 4).tolist() == [0, 1, 2, 5, 4, 3, 9, 10, 11, 8, 7, 6]
+
+
+ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_zigzag, pin_pool, pin_scan_dual,
             pin_scan_closed_forms, pin_bissd_dual, pin_bissd_flip_equivariance, pin_bissd_review,
             pin_tesa_golden, pin_tesa_tiling, pin_tesa_block_mask, pin_tesa_special]

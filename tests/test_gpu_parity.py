@@ -27,7 +27,7 @@ def _cuda():
 # index maps: bit exact
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("grid", [(2, 2, 3), (4, 8, 8), (3, 5, 7), (128, 32, 32), (1, 1, 1), (32, 48, 48)])
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 @pytest.mark.parametrize("flip", [False, True])
 def test_rms_map_bit_exact(grid, mode, flip):
     T, H, W = grid
@@ -61,13 +61,13 @@ def _bissd_case(cfg, mode, pool, chunk=None, heads=None, seed=0):
     return rel_err(got, ref)
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 def test_bissd_tiny_fp32(mode):
     cfg = workloads.CONFIGS["tiny"]
     assert _bissd_case(cfg, mode, cfg.review) <= TOL["f32"]
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 def test_bissd_tiny_no_review(mode):
     cfg = workloads.CONFIGS["tiny"]
     assert _bissd_case(cfg, mode, None) <= TOL["f32"]
@@ -88,7 +88,7 @@ def test_bissd_long_memory_fp32():
 def test_bissd_ragged_and_groups():
     # 105 tokens (not a multiple of the chunk), 4 heads in 2 B/C groups, batch 2
     cfg = workloads.CONFIGS["tiny"].with_(T=3, H=5, W=7, batch=2, nheads=4, ngroups=2, headdim=32, dstate=16)
-    for mode in range(4):
+    for mode in range(5):
         assert _bissd_case(cfg, mode, (3, 5, 7), chunk=32) <= TOL["f32"]
         assert _bissd_case(cfg, mode, None, chunk=32) <= TOL["f32"]
 
@@ -132,6 +132,13 @@ def test_bissd_512p_17s_bf16(mode):
 def test_bissd_512p_68s_bf16_full_size():
     cfg = workloads.CONFIGS["512p-68s"]
     assert _bissd_case(cfg, 3, cfg.review, heads=[5, 66]) <= TOL["bf16"]
+
+
+@pytest.mark.slow
+def test_bissd_512p_68s_zigzag_full_size():
+    # the zigzag comparison order on the 131k grid (gathered rows, review runs along W)
+    cfg = workloads.CONFIGS["512p-68s"]
+    assert _bissd_case(cfg, workloads.ZZ, cfg.review, heads=[17]) <= TOL["bf16"]
 
 
 @pytest.mark.slow

@@ -73,7 +73,7 @@ def test_ssd_tc_tma_rows_past_the_end():
     assert _run_ssd(cfg, inp, 1, (3, 4, 4), 256) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 def test_ssd_tc_review_runs(mode):
     # review boxes 4 or 8 tokens long on the scan's fastest axis: runs of 4 or 8 rows of a
     # sub-chunk share one box, and their sums are taken where the chunk states are; box
@@ -86,6 +86,16 @@ def test_ssd_tc_review_runs(mode):
     inp = workloads.generate(cfg, seed=9, parts=("ssd",))
     assert _run_ssd(cfg, inp, mode, (4, 4, 4), 512) <= TOL["bf16"]
     assert _run_ssd(cfg, inp, mode, (2, 4, 4), 384) <= TOL["bf16"]
+
+
+def test_ssd_tc_zigzag_odd_rows():
+    # the zigzag comparison order with an odd row count per frame (the row walking
+    # direction then flips parity from frame to frame), a ragged last chunk, batch 2
+    cfg = BF16_SSD.with_(T=3, H=5, W=24, batch=2, nheads=4)
+    inp = workloads.generate(cfg, seed=12, parts=("ssd",))
+    assert _run_ssd(cfg, inp, 4, None, 512) <= TOL["bf16"]
+    assert _run_ssd(cfg, inp, 4, (1, 5, 8), 256) <= TOL["bf16"]
+    assert _run_ssd(cfg, inp, 4, (3, 1, 3), 128) <= TOL["bf16"]
 
 
 def test_ssd_tc_review_extremes():

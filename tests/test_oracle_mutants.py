@@ -28,6 +28,8 @@ MUTANTS = [
     ("pool divides by a wrong count", "inv = 1.0 / ((double)pt * ph * pw);", "inv = 1.0 / ((double)pt * ph);"),
     ("pooled grid unrolled in grid order", "if (review) oracle_rms_sequence(Tp, Hp, Wp, mode, 0, porder);",
      "if (review) oracle_rms_sequence(Tp, Hp, Wp, 0, 0, porder);"),
+    ("zigzag rows all walked the same way", "const int w = (row % 2 == 0) ? j : W - 1 - j;", "const int w = j;"),
+    ("zigzag odd frames not reversed", "const int h = (t % 2 == 0) ? i : H - 1 - i;", "const int h = i;"),
     ("softmax without 1/sqrt(d)", "const double scale = 1.0 / sqrt((double)d);", "const double scale = 1.0;"),
     ("window boundaries at -shift", "for (int b = s; b < Lx; b += S) starts[n++] = b;",
      "for (int b = (S - s) % S; b < Lx; b += S) starts[n++] = b;"),

@@ -38,7 +38,8 @@ import torch
 
 # scan-mode codes shared by every layer of the stack
 SR, SC, TR, TC = 0, 1, 2, 3
-MODE_NAMES = {SR: "spatial-row", SC: "spatial-column", TR: "temporal-row", TC: "temporal-column"}
+ZZ = 4  # the zigzag scan the pages compare RMS against (a comparison order, not an RMS mode)
+MODE_NAMES = {SR: "spatial-row", SC: "spatial-column", TR: "temporal-row", TC: "temporal-column", ZZ: "zigzag"}
 
 
 @dataclass(frozen=True)
