@@ -224,11 +224,12 @@ def run_mate(args, cfg, rank, world, dist):
     sdims = api.ssd_dims(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, cfg.ngroups, cfg.chunk, cfg.torch_dtype)
     adims = api.attn_dims(cfg.batch, cfg.attn_heads, cfg.attn_dim, cfg.torch_dtype)
 
-    def step(src, o_ssd, o_att, workspace):
+    def step(src, o_ssd, o_att, workspace, strm=None):
+        strm = strm or stream
         api.mate_bissd_fwd(src["x"], src["dt"], src["A"], src["B"], src["C"], src["D"], cfg.T, cfg.H, cfg.W, mode,
-                           cfg.review, o_ssd, sdims, workspace, stream)
+                           cfg.review, o_ssd, sdims, workspace, strm)
         api.tesa_fwd(src["q"], src["k"], src["v"], cfg.T, cfg.H, cfg.W, cfg.Tw, cfg.Sw, cfg.shift, o_att, adims,
-                     stream)
+                     strm)
 
     # phase events recorded through the library's enqueue-time hook
     marks = []
@@ -290,37 +291,65 @@ def run_mate(args, cfg, rank, world, dist):
     phase_launch_avg = {k: sum(v) / len(v) for k, v in phase_ms.items()}
     launches_per_step = {k: len(v) / args.steps for k, v in phase_ms.items()}
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every step copies its
+    # inputs from pinned host memory and its outputs back. Steps are pipelined over
+    # three streams (copies in, compute, copies out) and two sets of device buffers,
+    # as a serving loop would run them: step i's inputs travel while step i-1
+    # computes and step i-2's outputs travel back.
     e2e = None
     if not args.no_e2e:
         pinned = {k: v.pin_memory() for k, v in host.items()}
-        h_ssd = torch.empty(out_ssd.shape, dtype=out_ssd.dtype).pin_memory()
-        h_att = torch.empty(out_att.shape, dtype=out_att.dtype).pin_memory()
+        h_out = [(torch.empty(out_ssd.shape, dtype=out_ssd.dtype).pin_memory(),
+                  torch.empty(out_att.shape, dtype=out_att.dtype).pin_memory()) for _ in range(2)]
         h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-        d2h = h_ssd.numel() * h_ssd.element_size() + h_att.numel() * h_att.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in h_out[0])
+        dsets = [d, {k: torch.empty_like(v) for k, v in d.items()}]
+        osets = [(out_ssd, out_att), (torch.empty_like(out_ssd), torch.empty_like(out_att))]
+        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        started = [False, False]
 
-        def e2e_step():
-            for k_, v_ in pinned.items():
-                d[k_].copy_(v_, non_blocking=True)
-            step(d, out_ssd, out_att, ws)
-            h_ssd.copy_(out_ssd, non_blocking=True)
-            h_att.copy_(out_att, non_blocking=True)
+        def e2e_step(i):
+            j = i % 2
+            if started[j]:
+                s_in.wait_event(ev_cmp[j])    # step i-2 has read this input set
+            with torch.cuda.stream(s_in):
+                for k_, v_ in pinned.items():
+                    dsets[j][k_].copy_(v_, non_blocking=True)
+            ev_in[j].record(s_in)
+            s_cmp.wait_event(ev_in[j])
+            if started[j]:
+                s_cmp.wait_event(ev_out[j])   # step i-2's outputs have left this set
+            step(dsets[j], osets[j][0], osets[j][1], ws, s_cmp)
+            ev_cmp[j].record(s_cmp)
+            s_out.wait_event(ev_cmp[j])
+            with torch.cuda.stream(s_out):
+                h_out[j][0].copy_(osets[j][0], non_blocking=True)
+                h_out[j][1].copy_(osets[j][1], non_blocking=True)
+            ev_out[j].record(s_out)
+            started[j] = True
 
-        for _ in range(min(args.warmup, 2)):
-            e2e_step()
+        k_e2e = max(1, min(args.steps, args.e2e_steps))
+        for i in range(min(args.warmup, 2)):
+            e2e_step(i)
         barrier()
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        k_e2e = max(1, min(args.steps, args.e2e_steps))
-        e0.record(stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)
+        for i in range(k_e2e):
+            e2e_step(i)
+        s_in.wait_event(ev_out[(k_e2e - 1) % 2])
+        s_in.wait_event(ev_out[k_e2e % 2])
+        e1.record(s_in)
         torch.cuda.synchronize()
         te = max_over_ranks(e0.elapsed_time(e1) / k_e2e, dist, dev)
         e2e = {"value": job_throughput(cfg.tokens, world, te), "unit": "Mtokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e,
+               "pipelined": "copies in, compute and copies out of consecutive steps overlap (3 streams)"}
+        del dsets, osets, h_out
 
     result = None
     if rank == 0:
