@@ -1047,14 +1047,16 @@ done:
 // ---------------------------------------------------------------------------
 // state_chain: one thread per eight consecutive elements of the 64 x 64 state
 // (one 16-byte vector). The chunk states are stored as bf16; the chain itself
-// runs in fp32, with the loads of kAhead chunks in flight ahead of it.
-// grid: (4096 / 8 / 256, nh * batch, 2 directions)
+// runs in fp32, with the loads of kAhead chunks in flight ahead of it. Three CTAs
+// per SM, so that the 320 CTAs of an 80-head grid all run at once (no tail wave).
+// grid: (4096 / 8 / kChainThreads, nh * batch, 2 directions)
 // ---------------------------------------------------------------------------
-constexpr int kAhead = 16;
+constexpr int kAhead = 8;
+constexpr int kChainThreads = 256;
 
-__global__ void __launch_bounds__(256) ssd_state_chain_kernel(SsdArgs a)
+__global__ void __launch_bounds__(kChainThreads, 3) ssd_state_chain_kernel(SsdArgs a)
 {
-    const int e8 = (blockIdx.x * 256 + threadIdx.x) * 8;  // first of this thread's 8 elements
+    const int e8 = (blockIdx.x * kChainThreads + threadIdx.x) * 8;  // first of this thread's 8 elements
     const int hb = blockIdx.y, dir = blockIdx.z;
     const int h = hb % a.nh, b = hb / a.nh;
     const int nc = a.nchunks;
@@ -1190,7 +1192,7 @@ cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s)
     }
     {
         Phase ph(MATE_PHASE_STATE_PASS, s);
-        ssd_state_chain_kernel<<<dim3(4096 / 8 / 256, a.nh * a.batch, 2), 256, 0, s>>>(a);
+        ssd_state_chain_kernel<<<dim3(4096 / 8 / kChainThreads, a.nh * a.batch, 2), kChainThreads, 0, s>>>(a);
     }
     // chunk_out is persistent: two CTAs per SM walk the (head, chunk, batch) items
     int dev = 0, nsm = 148;
