@@ -588,22 +588,23 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (!mma_wait(bar, mma_phase, a.err, abort_flag)) goto cleanup;
 
-        // row r of M: S columns 64g .. 64g+63 times the decay factors, as bf16 pairs into
-        // TMEM columns 0..31 (g = 0) or 96..127 (g = 1) of R, over S columns this thread
-        // has already read; the output MMA reads M from there as its A operand.
+        // row r of M: the thread's S columns, 16 of each 32-column block b (columns
+        // 32b + 16g ..), times the decay factors; each warp's diagonal block is thus
+        // split evenly between the row's two threads. The bf16 pairs of block b go to
+        // TMEM columns 32(b/2) + 16g + 8(b%2) of R (columns 0-63, S columns this thread
+        // has already read), where the output MMA reads M as its A operand.
         {
             const float ff = __expf(ci - rmid), fb = __expf(rmid - ei);
             const int wq = warp & 3;  // this warp's rows are 32*wq .. 32*wq + 31
-            uint32_t mp[2][16];       // the packed row half, 16 TMEM columns at a time
 #pragma unroll
             for (int qp = 0; qp < 4; qp += 2) {
-                uint32_t raw2[2][16];  // two 16-column TMEM loads per wait
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp), raw2[0]);
-                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 64 * g + 16 * qp + 16), raw2[1]);
+                uint32_t raw2[2][16], mp[2][8];  // two 16-column TMEM loads per wait
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * qp + 16 * g), raw2[0]);
+                tc::tmem_ld16(tc::tmem_addr(tR, lane_base, 32 * qp + 32 + 16 * g), raw2[1]);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int j0 = 64 * g + 16 * (qp + u);   // first of these 16 columns
+                    const int j0 = 32 * (qp + u) + 16 * g;   // first of these 16 columns
                     float sv[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sv[e] = __uint_as_float(raw2[u][e]);
@@ -652,12 +653,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                         }
                     }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) mp[qp >> 1][8 * u + e] = bf2(sv[2 * e], sv[2 * e + 1]);
+                    for (int e = 0; e < 8; ++e) mp[u][e] = bf2(sv[2 * e], sv[2 * e + 1]);
                 }
+                tc::tmem_st8(tc::tmem_addr(tR, lane_base, 16 * qp + 16 * g), mp[0]);
+                tc::tmem_st8(tc::tmem_addr(tR, lane_base, 16 * qp + 16 * g + 8), mp[1]);
             }
-            const uint32_t mcol = g ? 96u : 0u;
-            tc::tmem_st16(tc::tmem_addr(tR, lane_base, mcol), mp[0]);
-            tc::tmem_st16(tc::tmem_addr(tR, lane_base, mcol + 16), mp[1]);
             tc::tmem_wait_st();
         }
         {
@@ -676,9 +676,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::tc_fence_before();
         __syncthreads();
 
-        // Acc = M x + (R_f C) h_f^T + (R_b C) h_b^T -> TMEM R columns 32..95 (S there is
-        // consumed); M comes from TMEM (K-steps 0-3 at columns 0.., 4-7 at 96..)
-        const uint32_t tAcc = tR + 32;
+        // Acc = M x + (R_f C) h_f^T + (R_b C) h_b^T -> TMEM R columns 64..127 (S there is
+        // consumed); M comes from TMEM: K-step s (tokens 16s ..) is block s/2 of thread
+        // g = s%2, at column 32(s/4) + 16(s%2) + 8((s/2)%2)
+        const uint32_t tAcc = tR + 64;
         if (tid == 0) {
             tc::tc_fence_after();
             const uint32_t id_mx = tc::idesc_bf16(128, 64, 0, 1);
@@ -688,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint32_t hf = tc::smem_u32(sHf), hb = tc::smem_u32(sHb);
 #pragma unroll
             for (int s2 = 0; s2 < 8; ++s2)
-                tc::mma_bf16_tmem_a(tAcc, tR + (s2 < 4 ? 8 * s2 : 96 + 8 * (s2 - 4)),
+                tc::mma_bf16_tmem_a(tAcc, tR + 32 * (s2 >> 2) + 16 * (s2 & 1) + 8 * ((s2 >> 1) & 1),
                                     tc::sdesc_sw128(x0 + s2 * 2048, kTile, 1024), id_mx, s2 > 0);
 #pragma unroll
             for (int s2 = 0; s2 < 4; ++s2)
