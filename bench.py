@@ -470,6 +470,49 @@ def time_config(cfg, mode, steps, warmup, seed=0):
     return ms, phases
 
 
+def time_compose(cfg, steps, warmup, sample_rows=32):
+    """mate_compose_fwd on the grid's branch outputs: (tokens, nh*P) and
+    (tokens, th*td) rows to the model width. Device time from CUDA events,
+    the tensor-core fraction against the burst bf16 peak (a kernel timed on its
+    own), and the oracle timed on `sample_rows` rows, scaled to all rows."""
+    import torch
+
+    import linear_complexity_video_b200 as mate
+    import oracle
+
+    k1, k2, n = cfg.nheads * cfg.headdim, cfg.attn_heads * cfg.attn_dim, workloads.D_MODEL
+    host = workloads.generate_compose(cfg.tokens, k1, k2, n, seed=0)
+    d = {k: v.cuda() for k, v in host.items()}
+    out = torch.empty(cfg.tokens, n, dtype=torch.bfloat16, device="cuda")
+    for _ in range(warmup):
+        mate.compose(d["y_ma"], d["y_te"], d["w_ma"], d["w_te"], out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        mate.compose(d["y_ma"], d["y_te"], d["w_ma"], d["w_te"], out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    if mate.mate_last_error() != 0:
+        raise RuntimeError("device error word set")
+    ms = e0.elapsed_time(e1) / steps
+    flops = 2.0 * cfg.tokens * n * (k1 + k2)
+    nbytes = 2.0 * (cfg.tokens * (k1 + k2) + n * (k1 + k2) + cfg.tokens * n)
+    peaks, _ = load_peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    t0 = time.perf_counter()
+    oracle.get().compose(host["y_ma"][:sample_rows], host["y_te"][:sample_rows], host["w_ma"], host["w_te"])
+    t_or = (time.perf_counter() - t0) * cfg.tokens / sample_rows
+    del d, out
+    torch.cuda.empty_cache()
+    return {"report": "compose", "workload": cfg.name, "tokens": cfg.tokens, "k_ma": k1, "k_te": k2, "d_model": n,
+            "ms": round(ms, 4), "tflops": round(tf, 1), "tensor_peak_burst": float(peaks["bf16_tflops"]),
+            "tensor_frac": round(tf / float(peaks["bf16_tflops"]), 4),
+            "hbm_frac": round(nbytes / (ms / 1e3) / 1e9 / float(peaks["hbm_gbs"]), 4),
+            "mtokens_per_s": round(cfg.tokens / ms / 1e3, 2),
+            "oracle_s_scaled": round(t_or, 1), "oracle_sample_rows": sample_rows}
+
+
 def run_report(args):
     """Every bf16 grid in every scan order it lists, the headline grid in the
     zigzag comparison order, then the N sweep with a linearity fit. One JSON
@@ -500,6 +543,9 @@ def run_report(args):
                       "rms_scan": workloads.MODE_NAMES[cfg.modes[0]], "rms_ms_per_step": round(ms_rms, 4),
                       "zigzag_ms_per_step": round(ms_zz, 4), "zigzag_over_rms": round(ms_zz / ms_rms, 4),
                       "rms_phase_ms": ph_rms, "zigzag_phase_ms": ph_zz}), flush=True)
+    # the MATE composition (projections of both branches to the model width, summed) on
+    # the headline grid, against the tensor-core roofline; the oracle on a row sample
+    print(json.dumps(time_compose(cfg, args.steps, args.warmup)), flush=True)
     Ns, ts = [], []
     for cfg in workloads.sweep_configs():
         ms, phases = time_config(cfg, cfg.modes[0], args.steps, args.warmup)

@@ -231,6 +231,37 @@ int mate_bissd_fwd_noalloc(const void *x, const float *dt, const float *A, const
 int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, int Tw, int Sw,
              const int shift[3], void *out, const mate_attn_dims *d, void *stream);
 
+/* ---- MATE composition ---------------------------------------------------- */
+typedef struct {
+    int tokens;  /* rows M of every operand (all batch elements, grid order) */
+    int k_ma;    /* MA-branch channels (SSD heads x head dim, e.g. 80 x 64) */
+    int k_te;    /* TE-branch channels (TESA heads x head dim, e.g. 20 x 128) */
+    int d_model; /* output channels N (the block width, e.g. 2560) */
+    int dtype;   /* MATE_BF16 (the only storage the kernel takes) */
+} mate_compose_dims;
+
+/*
+ * MATE composition (paper review, section 三, MATE: the MA-branch and the
+ * TE-branch together replace self-attention). The pages give no combination
+ * rule; the two branch outputs have different widths, so each is projected
+ * to the model width and the projections are added:
+ *     out = y_ma W_ma^T + y_te W_te^T
+ * computed as one bf16 tensor-core GEMM over the concatenated K_MA + K_TE
+ * reduction with fp32 accumulation, rounded once to bf16.
+ *   y_ma : (tokens, k_ma)     bf16, row-major (the bi-SSD output viewed as rows)
+ *   y_te : (tokens, k_te)     bf16, row-major (the TESA output viewed as rows)
+ *   w_ma : (d_model, k_ma)    bf16, row-major (nn.Linear layout)
+ *   w_te : (d_model, k_te)    bf16, row-major
+ *   out  : (tokens, d_model)  bf16, row-major, caller-owned, must not overlap
+ *          the inputs
+ * All pointers device memory, 16-byte aligned. k_ma and k_te are multiples of
+ * 64 (either may be 0, not both), d_model a multiple of 64, tokens > 0.
+ * Returns MATE_OK, MATE_ERR_INVALID_ARG (bad pointers, sizes or overlap),
+ * MATE_ERR_UNSUPPORTED (other dtype or sizes) or MATE_ERR_CUDA.
+ */
+int mate_compose_fwd(const void *y_ma, const void *y_te, const void *w_ma, const void *w_te, void *out,
+                     const mate_compose_dims *d, void *stream);
+
 /*
  * Debug export of the scan order the kernels use: out_dev[n] = grid offset
  * of the n-th token of the scan (flip != 0: of the flipped scan). out_dev
@@ -277,6 +308,7 @@ int mate_last_error(void *stream);
 #define MATE_PHASE_STATE_PASS 4  /* chain chunk states -> state entering each chunk */
 #define MATE_PHASE_CHUNK_OUT 5   /* outputs of every chunk, both directions         */
 #define MATE_PHASE_TESA 6        /* windowed attention                             */
+#define MATE_PHASE_COMPOSE 7     /* mate_compose_fwd's projection GEMM              */
 
 /*
  * Optional enqueue-time hook, for timing phases with events on the caller's

@@ -37,11 +37,13 @@ EXPORTS = (
     "mate_set_phase_hook",
     "mate_kernel_launches",
     "mate_bissd_fwd_noalloc",
+    "mate_compose_fwd",
 )
 
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
-PHASES = {1: "review_pool", 2: "review_scan", 3: "chunk_state", 4: "state_pass", 5: "chunk_out", 6: "tesa"}
+PHASES = {1: "review_pool", 2: "review_scan", 3: "chunk_state", 4: "state_pass", 5: "chunk_out", 6: "tesa",
+          7: "compose"}
 PHASE_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
 
 
@@ -53,6 +55,11 @@ class mate_ssd_dims(ctypes.Structure):
 
 class mate_attn_dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("nheads", ctypes.c_int), ("headdim", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+class mate_compose_dims(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_int), ("k_ma", ctypes.c_int), ("k_te", ctypes.c_int), ("d_model", ctypes.c_int),
                 ("dtype", ctypes.c_int)]
 
 
@@ -92,6 +99,8 @@ def load() -> ctypes.CDLL:
     L.mate_status_string.restype = ctypes.c_char_p
     L.mate_debug_fastdiv.argtypes = [_vp, _vp, ctypes.c_size_t, ctypes.c_uint32]
     L.mate_debug_fastdiv.restype = ctypes.c_int
+    L.mate_compose_fwd.argtypes = [_vp] * 5 + [ctypes.POINTER(mate_compose_dims), _vp]
+    L.mate_compose_fwd.restype = ctypes.c_int
     L.mate_version.argtypes = []
     L.mate_version.restype = ctypes.c_int
     L.mate_set_phase_hook.argtypes = [PHASE_HOOK, ctypes.c_void_p]

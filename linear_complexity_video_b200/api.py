@@ -14,7 +14,7 @@ from typing import Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import MATE_BF16, MATE_DIR_BI, MATE_F32, check, mate_attn_dims, mate_ssd_dims
+from ._lib import MATE_BF16, MATE_DIR_BI, MATE_F32, check, mate_attn_dims, mate_compose_dims, mate_ssd_dims
 
 _DT = {torch.float32: MATE_F32, torch.bfloat16: MATE_BF16}
 
@@ -86,6 +86,12 @@ def tesa_fwd(q, k, v, T, H, W, Tw, Sw, shift, out, dims: mate_attn_dims, stream=
     check("tesa_fwd", rc)
 
 
+def mate_compose_fwd(y_ma, y_te, w_ma, w_te, out, dims: mate_compose_dims, stream=None) -> None:
+    rc = _lib.load().mate_compose_fwd(_ptr(y_ma), _ptr(y_te), _ptr(w_ma), _ptr(w_te), _ptr(out), ctypes.byref(dims),
+                                      _stream_handle(stream))
+    check("mate_compose_fwd", rc)
+
+
 def mate_debug_rms_map(T, H, W, scan_mode, flip, out, stream=None) -> None:
     check("mate_debug_rms_map",
           _lib.load().mate_debug_rms_map(T, H, W, scan_mode, int(flip), _ptr(out), _stream_handle(stream)))
@@ -145,6 +151,26 @@ def tesa(q, k, v, Tw: int, Sw: int, shift=(0, 0, 0), out: Optional[torch.Tensor]
     if out is None:
         out = torch.empty_like(q)
     tesa_fwd(q, k, v, T, H, W, Tw, Sw, shift, out, attn_dims(b, nh, d, q.dtype), stream)
+    return out
+
+
+def compose(y_ma, y_te, w_ma, w_te, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """MATE composition: out = y_ma w_ma^T + y_te w_te^T (bf16). y_ma: (..., k_ma), the bi-SSD
+    output with its heads flattened; y_te: (..., k_te), the TESA output likewise; w_ma: (d_model,
+    k_ma), w_te: (d_model, k_te). Returns (..., d_model)."""
+    for t, n in ((y_ma, "y_ma"), (y_te, "y_te"), (w_ma, "w_ma"), (w_te, "w_te")):
+        _require(t, n, torch.bfloat16)
+    lead = y_ma.shape[:-1]
+    if y_te.shape[:-1] != lead:
+        raise ValueError("y_ma and y_te must cover the same tokens")
+    M = 1
+    for s in lead:
+        M *= int(s)
+    N = int(w_ma.shape[0])
+    if out is None:
+        out = torch.empty(*lead, N, dtype=torch.bfloat16, device=y_ma.device)
+    dims = mate_compose_dims(M, int(y_ma.shape[-1]), int(y_te.shape[-1]), N, MATE_BF16)
+    mate_compose_fwd(y_ma, y_te, w_ma, w_te, out, dims, stream)
     return out
 
 

@@ -93,6 +93,15 @@ struct TesaArgs {
     int *err;                // device error word
 };
 
+// MATE composition: out (M x N) = y1 (M x K1) w1^T + y2 (M x K2) w2^T, bf16
+// row-major, w1 (N x K1) and w2 (N x K2) in the nn.Linear layout.
+struct ComposeArgs {
+    const void *y1, *y2, *w1, *w2;
+    void *out;
+    int M, N, K1, K2;
+    int *err;                // device error word
+};
+
 // Phase hook and launch counter (mate_set_phase_hook / mate_kernel_launches).
 void phase_mark(int phase, int is_end, cudaStream_t s);
 void count_launch();
@@ -126,6 +135,8 @@ cudaError_t launch_tesa_generic(const TesaArgs &a, cudaStream_t s);
 // tensor-core TESA path (bf16, head dim 128, 128-token windows)
 bool tesa_tc_supported(const TesaArgs &a);
 cudaError_t launch_tesa_tc(const TesaArgs &a, cudaStream_t s);
+bool compose_tc_supported(const ComposeArgs &a);
+cudaError_t launch_compose_tc(const ComposeArgs &a, cudaStream_t s);
 // tensor-core bi-SSD path (bf16, head dim 64, d_state 64, both directions)
 bool ssd_tc_supported(const SsdArgs &a);
 cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s);

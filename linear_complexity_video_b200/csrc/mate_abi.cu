@@ -297,6 +297,37 @@ int tesa_fwd(const void *q, const void *k, const void *v, int T, int H, int W, i
     return err == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
 }
 
+int mate_compose_fwd(const void *y_ma, const void *y_te, const void *w_ma, const void *w_te, void *out,
+                     const mate_compose_dims *d, void *stream)
+{
+    if (!d) return MATE_ERR_INVALID_ARG;
+    if (d->tokens <= 0 || d->k_ma < 0 || d->k_te < 0 || d->d_model <= 0 || d->k_ma + d->k_te <= 0)
+        return MATE_ERR_INVALID_ARG;
+    if (d->dtype != MATE_BF16) return MATE_ERR_UNSUPPORTED;
+    ComposeArgs a;
+    a.M = d->tokens;
+    a.N = d->d_model;
+    a.K1 = d->k_ma;
+    a.K2 = d->k_te;
+    if (!compose_tc_supported(a)) return MATE_ERR_UNSUPPORTED;
+    if (!out || (a.K1 && (!y_ma || !w_ma)) || (a.K2 && (!y_te || !w_te))) return MATE_ERR_INVALID_ARG;
+    const void *ptrs[5] = {y_ma, y_te, w_ma, w_te, out};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return MATE_ERR_INVALID_ARG;
+    const size_t ob = (size_t)a.M * a.N * 2;
+    if ((a.K1 && (overlaps(out, ob, y_ma, (size_t)a.M * a.K1 * 2) || overlaps(out, ob, w_ma, (size_t)a.N * a.K1 * 2))) ||
+        (a.K2 && (overlaps(out, ob, y_te, (size_t)a.M * a.K2 * 2) || overlaps(out, ob, w_te, (size_t)a.N * a.K2 * 2))))
+        return MATE_ERR_INVALID_ARG;
+    a.y1 = y_ma;
+    a.y2 = y_te;
+    a.w1 = w_ma;
+    a.w2 = w_te;
+    a.out = out;
+    a.err = error_word_ptr();
+    if (!a.err) return MATE_ERR_CUDA;
+    return launch_compose_tc(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
 int mate_debug_rms_map(int T, int H, int W, int scan_mode, int flip, int32_t *out_dev, void *stream)
 {
     if (T <= 0 || H <= 0 || W <= 0 || scan_mode < 0 || scan_mode > MATE_SCAN_ZZ || !out_dev)

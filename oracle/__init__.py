@@ -63,8 +63,9 @@ class Oracle:
         L.oracle_bissd.argtypes = [ctypes.c_int] * 8 + [_f64p] * 6 + [ctypes.c_int, _intp, _f64p]
         L.oracle_tesa_window_ids.argtypes = [ctypes.c_int] * 5 + [_intp, _i32p]
         L.oracle_tesa.argtypes = [ctypes.c_int] * 6 + [_f64p] * 3 + [ctypes.c_int] * 2 + [_intp, _f64p]
+        L.oracle_compose.argtypes = [ctypes.c_int64] + [ctypes.c_int] * 3 + [_f64p] * 5
         for f in ("oracle_unroll", "oracle_rms_sequence", "oracle_avg_pool", "oracle_ssd_scan",
-                  "oracle_bissd", "oracle_tesa_window_ids", "oracle_tesa"):
+                  "oracle_bissd", "oracle_tesa_window_ids", "oracle_tesa", "oracle_compose"):
             getattr(L, f).restype = ctypes.c_int
 
     # ---- Rotary Major Scan -------------------------------------------------
@@ -140,6 +141,24 @@ class Oracle:
         if rc < 0:
             raise ValueError(f"oracle_tesa rc={rc}")
         return out
+
+
+    # ---- MATE composition --------------------------------------------------
+    def compose(self, y_ma, y_te, w_ma, w_te) -> np.ndarray:
+        """out = y_ma w_ma^T + y_te w_te^T. y_ma: (..., K1), y_te: (..., K2) over the same
+        leading shape; w_ma: (N, K1), w_te: (N, K2). Returns (..., N)."""
+        y1, y2, w1, w2 = map(_f64, (y_ma, y_te, w_ma, w_te))
+        lead = y1.shape[:-1]
+        K1, K2, N = y1.shape[-1], y2.shape[-1], w1.shape[0]
+        M = int(np.prod(lead)) if lead else 1
+        y1 = np.ascontiguousarray(y1.reshape(M, K1))
+        y2 = np.ascontiguousarray(y2.reshape(M, K2))
+        out = np.empty((M, N), dtype=np.float64)
+        rc = self.lib.oracle_compose(M, K1, K2, N, _ptr(y1, _f64p), _ptr(y2, _f64p), _ptr(w1, _f64p),
+                                     _ptr(w2, _f64p), _ptr(out, _f64p))
+        if rc:
+            raise ValueError(f"oracle_compose rc={rc}")
+        return out.reshape(*lead, N)
 
 
 _default: Optional[Oracle] = None

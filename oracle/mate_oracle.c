@@ -39,6 +39,8 @@
  *      window, no mask inside a window, no position bias.
  *   R6 Zigzag scan (named, not defined, by the pages): the 3D boustrophedon
  *      of oracle_zigzag, used only as the comparison order.
+ *   R7 MATE composition: the two branch outputs (different widths) are each
+ *      projected to the model width and added; no gate, no bias.
  */
 #include <math.h>
 #include <stdint.h>
@@ -432,4 +434,27 @@ int oracle_tesa(int batch, int T, int H, int W, int nh, int d,
             }
     free(win); free(count); free(members); free(fill);
     return err ? ORACLE_ENOMEM : nwin;
+}
+
+/* MATE composition ([Review] section 三, MATE: the MA-branch and the TE-branch
+ * together replace self-attention; reading R7): the block output is the sum of
+ * the two branches projected to the model width,
+ *     out[i][n] = sum_k y1[i][k] w1[n][k] + sum_k y2[i][k] w2[n][k],
+ * every row of y1 (M x K1) and y2 (M x K2) against every row of w1 (N x K1)
+ * and w2 (N x K2), each sum in order of k, the two sums added last. */
+int oracle_compose(int64_t M, int K1, int K2, int N, const double *y1, const double *y2, const double *w1,
+                   const double *w2, double *out)
+{
+    if (M < 0 || K1 < 0 || K2 < 0 || N <= 0 || !out || (K1 && (!y1 || !w1)) || (K2 && (!y2 || !w2)))
+        return ORACLE_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < M; ++i) {
+        for (int n = 0; n < N; ++n) {
+            double s1 = 0.0, s2 = 0.0;
+            for (int k = 0; k < K1; ++k) s1 += y1[i * K1 + k] * w1[(int64_t)n * K1 + k];
+            for (int k = 0; k < K2; ++k) s2 += y2[i * K2 + k] * w2[(int64_t)n * K2 + k];
+            out[i * N + n] = s1 + s2;
+        }
+    }
+    return ORACLE_OK;
 }

@@ -368,6 +368,25 @@ def pin_zigzag(o):
     assert o.rms_sequence(2, 2, 3, 4).tolist() == [0, 1, 2, 5, 4, 3, 9, 10, 11, 8, 7, 6]
 
 
-ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_zigzag, pin_pool, pin_scan_dual,
+def pin_compose(o):
+    """MATE composition (reading R7): a tiny case written out by hand, the
+    two-part split (each branch alone, zeros in the other, adds up to the
+    whole), and agreement with numpy's float64 matmul on a random case."""
+    y1, y2 = np.array([[2.0]]), np.array([[3.0]])
+    w1, w2 = np.array([[1.0], [4.0]]), np.array([[5.0], [6.0]])
+    assert o.compose(y1, y2, w1, w2).tolist() == [[2 * 1 + 3 * 5, 2 * 4 + 3 * 6]]
+    rng = np.random.default_rng(4)
+    y1, y2 = rng.standard_normal((2, 3, 5, 24)), rng.standard_normal((2, 3, 5, 16))
+    w1, w2 = rng.standard_normal((7, 24)), rng.standard_normal((7, 16))
+    full = o.compose(y1, y2, w1, w2)
+    assert full.shape == (2, 3, 5, 7)
+    parts = o.compose(y1, np.zeros_like(y2), w1, w2) + o.compose(np.zeros_like(y1), y2, w1, w2)
+    _close(full, parts, 1e-12, "the two branches do not add up")
+    _close(full, y1 @ w1.T + y2 @ w2.T, 1e-12, "composition against numpy matmul")
+    # each projection is applied to its own branch: swapping the weights changes the result
+    assert not np.allclose(full, y1 @ w1.T + y2 @ (w2[::-1]).T)
+
+
+ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_zigzag, pin_compose, pin_pool, pin_scan_dual,
             pin_scan_closed_forms, pin_bissd_dual, pin_bissd_flip_equivariance, pin_bissd_review,
             pin_tesa_golden, pin_tesa_tiling, pin_tesa_block_mask, pin_tesa_special]

@@ -199,3 +199,27 @@ def test_fastdiv_rejects_out_of_range():
     assert L.mate_debug_fastdiv(n.ctypes.data, q.ctypes.data, 1, 1 << 31) == _lib.MATE_ERR_INVALID_ARG
     assert L.mate_debug_fastdiv(None, None, 1, 3) == _lib.MATE_ERR_INVALID_ARG
     assert q[0] == 0
+
+
+def test_compose_rejects_bad_arguments():
+    """mate_compose_fwd checks its sizes, dtype and pointers before any CUDA call."""
+    L = mate.load()
+    p = ctypes.c_void_p(256)
+    ok = _lib.mate_compose_dims(128, 5120, 2560, 2560, _lib.MATE_BF16)
+    assert L.mate_compose_fwd(p, p, p, p, p, None, None) == _lib.MATE_ERR_INVALID_ARG
+    for bad in [(0, 64, 64, 64), (128, 0, 0, 64), (128, 64, 64, 0), (128, -64, 64, 64)]:
+        d = _lib.mate_compose_dims(*bad, _lib.MATE_BF16)
+        assert L.mate_compose_fwd(p, p, p, p, p, ctypes.byref(d), None) == _lib.MATE_ERR_INVALID_ARG, bad
+    for bad in [(128, 5000, 2560, 2560), (128, 5120, 2560, 2500), (128, 5120, 100, 2560)]:
+        d = _lib.mate_compose_dims(*bad, _lib.MATE_BF16)
+        assert L.mate_compose_fwd(p, p, p, p, p, ctypes.byref(d), None) == _lib.MATE_ERR_UNSUPPORTED, bad
+    d = _lib.mate_compose_dims(128, 5120, 2560, 2560, _lib.MATE_F32)
+    assert L.mate_compose_fwd(p, p, p, p, p, ctypes.byref(d), None) == _lib.MATE_ERR_UNSUPPORTED
+    assert L.mate_compose_fwd(p, p, p, p, None, ctypes.byref(ok), None) == _lib.MATE_ERR_INVALID_ARG
+    assert L.mate_compose_fwd(None, p, p, p, p, ctypes.byref(ok), None) == _lib.MATE_ERR_INVALID_ARG
+    q = ctypes.c_void_p(264)  # 8-byte aligned only
+    assert L.mate_compose_fwd(q, p, p, p, p, ctypes.byref(ok), None) == _lib.MATE_ERR_INVALID_ARG
+    # one branch absent: its pointers may be null
+    one = _lib.mate_compose_dims(128, 0, 2560, 2560, _lib.MATE_BF16)
+    r = ctypes.c_void_p(1 << 40)
+    assert L.mate_compose_fwd(None, p, None, r, None, ctypes.byref(one), None) == _lib.MATE_ERR_INVALID_ARG

@@ -30,6 +30,9 @@ MUTANTS = [
      "if (review) oracle_rms_sequence(Tp, Hp, Wp, 0, 0, porder);"),
     ("zigzag rows all walked the same way", "const int w = (row % 2 == 0) ? j : W - 1 - j;", "const int w = j;"),
     ("zigzag odd frames not reversed", "const int h = (t % 2 == 0) ? i : H - 1 - i;", "const int h = i;"),
+    ("composition drops the TE branch", "out[i * N + n] = s1 + s2;", "out[i * N + n] = s1;"),
+    ("composition reads w1 transposed", "s1 += y1[i * K1 + k] * w1[(int64_t)n * K1 + k];",
+     "s1 += y1[i * K1 + k] * w1[(int64_t)(k % N) * K1 + n % K1];"),
     ("softmax without 1/sqrt(d)", "const double scale = 1.0 / sqrt((double)d);", "const double scale = 1.0;"),
     ("window boundaries at -shift", "for (int b = s; b < Lx; b += S) starts[n++] = b;",
      "for (int b = (S - s) % S; b < Lx; b += S) starts[n++] = b;"),

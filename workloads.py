@@ -99,6 +99,25 @@ CONFIGS: Dict[str, Config] = {
 HEADLINE = "512p-68s"
 
 
+# model width of the MATE block ([Review] 5.1: embedding width 2560)
+D_MODEL = 2560
+
+
+def generate_compose(tokens: int, k_ma: int, k_te: int, d_model: int = D_MODEL, seed: int = 0,
+                     dtype=torch.bfloat16) -> Dict[str, torch.Tensor]:
+    """Inputs of the MATE composition on the host: the two branch outputs as
+    rows (y_ma ~ N(0, 1), y_te ~ N(0, 1)) and random-init projections in the
+    nn.Linear layout, w ~ N(0, 1 / (k_ma + k_te)) (so that out has unit scale),
+    from a generator seeded with seed + 2 in the order y_ma, y_te, w_ma, w_te."""
+    g = torch.Generator().manual_seed(seed + 2)
+    scale = 1.0 / math.sqrt(max(k_ma + k_te, 1))
+    y_ma = torch.randn(tokens, k_ma, generator=g)
+    y_te = torch.randn(tokens, k_te, generator=g)
+    w_ma = torch.randn(d_model, k_ma, generator=g) * scale
+    w_te = torch.randn(d_model, k_te, generator=g) * scale
+    return {k: v.to(dtype) for k, v in dict(y_ma=y_ma, y_te=y_te, w_ma=w_ma, w_te=w_te).items()}
+
+
 def sweep_configs():
     """N from 8k to 131k tokens at H=W=32 with the 131k grid's other settings."""
     base = CONFIGS[HEADLINE]
