@@ -513,6 +513,75 @@ def time_compose(cfg, steps, warmup, sample_rows=32):
             "oracle_s_scaled": round(t_or, 1), "oracle_sample_rows": sample_rows}
 
 
+def time_frontend(cfg, steps, warmup):
+    """mate_frontend_fwd on the grid (d_model 2560 to z, x, B, C, dt): device time
+    from CUDA events, the split by phase from the phase hook, the in_proj GEMMs
+    against the burst bf16 peak and the conv against the HBM peak (its
+    algorithmic bytes: the conv channels read once and written once)."""
+    import torch
+
+    import linear_complexity_video_b200 as mate
+    from linear_complexity_video_b200 import _lib
+
+    host = workloads.generate_frontend(cfg, seed=0)
+    d = {k: v.cuda() for k, v in host.items()}
+    mode = cfg.modes[0]
+
+    def call():
+        return mate.frontend(d["u"], d["w_in"], d["conv_w"], d["conv_b"], d["dt_bias"], mode, cfg.nheads,
+                             cfg.headdim, cfg.ngroups, cfg.dstate)
+
+    for _ in range(warmup):
+        outs = call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        outs = call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    marks, stream = [], torch.cuda.current_stream()
+
+    def hook(ph, is_end, strm, user):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        marks.append((ph, is_end, ev))
+
+    L = mate.load()
+    h = _lib.PHASE_HOOK(hook)
+    L.mate_set_phase_hook(h, None)
+    outs = call()
+    torch.cuda.synchronize()
+    L.mate_set_phase_hook(_lib.PHASE_HOOK(), None)
+    if mate.mate_last_error() != 0:
+        raise RuntimeError("device error word set")
+    phases, opened = {}, {}
+    for ph, is_end, ev in marks:
+        if not is_end:
+            opened[ph] = ev
+        else:
+            name = _lib.PHASES[ph]
+            phases[name] = phases.get(name, 0.0) + opened.pop(ph).elapsed_time(ev)
+    d_inner = cfg.nheads * cfg.headdim
+    dc = d_inner + 2 * cfg.ngroups * cfg.dstate
+    rows = d_inner + dc + cfg.nheads
+    flops = 2.0 * cfg.tokens * workloads.D_MODEL * rows
+    conv_bytes = 2.0 * cfg.tokens * dc * 2
+    peaks, _ = load_peaks()
+    proj = phases.get("front_proj", 0.0)
+    conv = phases.get("front_conv", 0.0)
+    del d, outs
+    torch.cuda.empty_cache()
+    return {"report": "frontend", "workload": cfg.name, "scan": workloads.MODE_NAMES[mode], "tokens": cfg.tokens,
+            "d_model": workloads.D_MODEL, "in_proj_rows": rows, "ms": round(ms, 4),
+            "phase_ms": {k: round(v, 4) for k, v in phases.items()},
+            "in_proj_tflops": round(flops / (proj / 1e3) / 1e12, 1) if proj else None,
+            "in_proj_tensor_frac": round(flops / (proj / 1e3) / 1e12 / float(peaks["bf16_tflops"]), 4) if proj else None,
+            "conv_hbm_frac": round(conv_bytes / (conv / 1e3) / 1e9 / float(peaks["hbm_gbs"]), 4) if conv else None,
+            "mtokens_per_s": round(cfg.tokens / ms / 1e3, 2)}
+
+
 def run_report(args):
     """Every bf16 grid in every scan order it lists, the headline grid in the
     zigzag comparison order, then the N sweep with a linearity fit. One JSON
@@ -546,6 +615,7 @@ def run_report(args):
     # the MATE composition (projections of both branches to the model width, summed) on
     # the headline grid, against the tensor-core roofline; the oracle on a row sample
     print(json.dumps(time_compose(cfg, args.steps, args.warmup)), flush=True)
+    print(json.dumps(time_frontend(cfg, args.steps, args.warmup)), flush=True)
     Ns, ts = [], []
     for cfg in workloads.sweep_configs():
         ms, phases = time_config(cfg, cfg.modes[0], args.steps, args.warmup)

@@ -262,6 +262,54 @@ typedef struct {
 int mate_compose_fwd(const void *y_ma, const void *y_te, const void *w_ma, const void *w_te, void *out,
                      const mate_compose_dims *d, void *stream);
 
+/* ---- MA-branch front-end ------------------------------------------------- */
+typedef struct {
+    int batch;
+    int d_model; /* block width (e.g. 2560) */
+    int nheads;  /* SSD heads; d_inner = nheads * headdim (e.g. 80 x 64) */
+    int headdim;
+    int ngroups; /* B/C groups */
+    int dstate;
+    int dtype;   /* MATE_BF16 (the only storage the kernels take) */
+} mate_frontend_dims;
+
+/*
+ * Workspace bytes mate_frontend_fwd needs (0 on bad or unsupported
+ * arguments): the in_proj outputs that the conv and dt steps read, bf16.
+ */
+size_t mate_frontend_workspace_bytes(int T, int H, int W, const mate_frontend_dims *d);
+
+/*
+ * MA-branch front-end: the input side of the Mamba2 block that produces the
+ * bi-SSD's inputs (paper review, section 三, MA-Branch item 1, bidirectional
+ * Mamba2; the pages give no more of the block, so this is the standard
+ * Mamba2 input side, with d_inner = nheads * headdim and dc = d_inner + 2 *
+ * ngroups * dstate conv channels):
+ *     [z | xBC_pre | dt_raw] = u W_in^T
+ *     xBC_n = SiLU(conv_b + sum_{k=0..3} conv_w[., k] * xBC_pre_{n-3+k})
+ *             along the scan order `scan_mode` (causal, depthwise, width 4,
+ *             positions before the first are zero); xBC = [x | B | C]
+ *     dt = softplus(dt_raw + dt_bias)
+ * The conv runs once, in the forward scan order; its result feeds both scan
+ * directions of mate_bissd_fwd. Everything stays in grid order.
+ *   u      : (batch, T, H, W, d_model)              bf16
+ *   w_in   : (d_inner + dc + nheads, d_model)       bf16 (nn.Linear layout,
+ *            rows z, then x, B, C, then dt)
+ *   conv_w : (dc, 4) fp32;  conv_b : (dc) fp32;  dt_bias : (nheads) fp32
+ *   z      : (batch, T, H, W, d_inner)              bf16 (the gate, for later)
+ *   x      : (batch, T, H, W, nheads, headdim)      bf16
+ *   dt     : (batch, T, H, W, nheads)               fp32
+ *   B, C   : (batch, T, H, W, ngroups, dstate)      bf16
+ * Device pointers; bf16 ones 16-byte aligned, fp32 ones 4-byte aligned;
+ * outputs caller-owned and disjoint from the inputs and the workspace.
+ * Supported: d_model a multiple of 64, d_inner and ngroups * dstate even,
+ * dc and nheads multiples of 8. Returns MATE_OK, MATE_ERR_INVALID_ARG,
+ * MATE_ERR_UNSUPPORTED, MATE_ERR_WORKSPACE or MATE_ERR_CUDA.
+ */
+int mate_frontend_fwd(const void *u, const void *w_in, const float *conv_w, const float *conv_b, const float *dt_bias,
+                      int T, int H, int W, int scan_mode, void *z, void *x, float *dt, void *B, void *C,
+                      const mate_frontend_dims *d, void *workspace, size_t ws_bytes, void *stream);
+
 /*
  * Debug export of the scan order the kernels use: out_dev[n] = grid offset
  * of the n-th token of the scan (flip != 0: of the flipped scan). out_dev
@@ -309,6 +357,9 @@ int mate_last_error(void *stream);
 #define MATE_PHASE_CHUNK_OUT 5   /* outputs of every chunk, both directions         */
 #define MATE_PHASE_TESA 6        /* windowed attention                             */
 #define MATE_PHASE_COMPOSE 7     /* mate_compose_fwd's projection GEMM              */
+#define MATE_PHASE_FRONT_PROJ 8  /* mate_frontend_fwd: one in_proj GEMM (3 per call) */
+#define MATE_PHASE_FRONT_CONV 9  /* mate_frontend_fwd: conv along the scan + SiLU   */
+#define MATE_PHASE_FRONT_DT 10   /* mate_frontend_fwd: softplus(dt + bias)          */
 
 /*
  * Optional enqueue-time hook, for timing phases with events on the caller's

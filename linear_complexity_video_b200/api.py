@@ -14,7 +14,8 @@ from typing import Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import MATE_BF16, MATE_DIR_BI, MATE_F32, check, mate_attn_dims, mate_compose_dims, mate_ssd_dims
+from ._lib import (MATE_BF16, MATE_DIR_BI, MATE_F32, check, mate_attn_dims, mate_compose_dims, mate_frontend_dims,
+                   mate_ssd_dims)
 
 _DT = {torch.float32: MATE_F32, torch.bfloat16: MATE_BF16}
 
@@ -172,6 +173,44 @@ def compose(y_ma, y_te, w_ma, w_te, out: Optional[torch.Tensor] = None, stream=N
     dims = mate_compose_dims(M, int(y_ma.shape[-1]), int(y_te.shape[-1]), N, MATE_BF16)
     mate_compose_fwd(y_ma, y_te, w_ma, w_te, out, dims, stream)
     return out
+
+
+def mate_frontend_workspace_bytes(T: int, H: int, W: int, dims: mate_frontend_dims) -> int:
+    return int(_lib.load().mate_frontend_workspace_bytes(T, H, W, ctypes.byref(dims)))
+
+
+def mate_frontend_fwd(u, w_in, conv_w, conv_b, dt_bias, T, H, W, scan_mode, z, x, dt, B, C,
+                      dims: mate_frontend_dims, workspace, stream=None) -> None:
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = _lib.load().mate_frontend_fwd(_ptr(u), _ptr(w_in), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), T, H, W,
+                                       scan_mode, _ptr(z), _ptr(x), _ptr(dt), _ptr(B), _ptr(C), ctypes.byref(dims),
+                                       _ptr(workspace), nbytes, _stream_handle(stream))
+    check("mate_frontend_fwd", rc)
+
+
+def frontend(u, w_in, conv_w, conv_b, dt_bias, scan_mode: int, nheads: int, headdim: int, ngroups: int, dstate: int,
+             stream=None):
+    """MA-branch front-end. u: (batch, T, H, W, d_model) bf16; w_in: (d_inner + dc + nheads, d_model)
+    bf16; conv_w: (dc, 4), conv_b: (dc), dt_bias: (nheads) fp32. Returns z, x, dt, B, C shaped as
+    mate_bissd_fwd and the gate take them."""
+    _require(u, "u", torch.bfloat16)
+    _require(w_in, "w_in", torch.bfloat16)
+    for t, n in ((conv_w, "conv_w"), (conv_b, "conv_b"), (dt_bias, "dt_bias")):
+        _require(t, n, torch.float32)
+    b, T, H, W, dm = u.shape
+    dims = mate_frontend_dims(b, dm, nheads, headdim, ngroups, dstate, MATE_BF16)
+    nbytes = mate_frontend_workspace_bytes(T, H, W, dims)
+    if nbytes == 0:
+        raise ValueError("unsupported front-end dims")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=u.device)
+    kw = dict(dtype=torch.bfloat16, device=u.device)
+    z = torch.empty(b, T, H, W, nheads * headdim, **kw)
+    x = torch.empty(b, T, H, W, nheads, headdim, **kw)
+    dt = torch.empty(b, T, H, W, nheads, dtype=torch.float32, device=u.device)
+    Bm = torch.empty(b, T, H, W, ngroups, dstate, **kw)
+    Cm = torch.empty(b, T, H, W, ngroups, dstate, **kw)
+    mate_frontend_fwd(u, w_in, conv_w, conv_b, dt_bias, T, H, W, scan_mode, z, x, dt, Bm, Cm, dims, ws, stream)
+    return z, x, dt, Bm, Cm
 
 
 def rms_map(T: int, H: int, W: int, scan_mode: int, flip: bool = False, device="cuda") -> torch.Tensor:

@@ -210,9 +210,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+// Any N that keeps rows 16-byte aligned: the B tiles past N load as zeros and the
+// output columns past N are clipped by the TMA store (a 64-column chunk that
+// starts past N is skipped).
 bool compose_tc_supported(const ComposeArgs &a)
 {
-    return a.M > 0 && a.N > 0 && a.N % 64 == 0 && a.K1 % kBK == 0 && a.K2 % kBK == 0 && a.K1 + a.K2 > 0;
+    return a.M > 0 && a.N > 0 && a.N % 8 == 0 && a.K1 % kBK == 0 && a.K2 % kBK == 0 && a.K1 + a.K2 > 0;
 }
 
 cudaError_t launch_compose_tc(const ComposeArgs &a, cudaStream_t s)
@@ -246,7 +249,7 @@ cudaError_t launch_compose_tc(const ComposeArgs &a, cudaStream_t s)
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const int grid = std::min(geo.tiles, std::max(nsm, 1));
-    Phase ph(MATE_PHASE_COMPOSE, s);
+    Phase ph(a.phase ? a.phase : MATE_PHASE_COMPOSE, s);
     compose_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma1, mb1, ma2, mb2, mo, geo, a.err);
     return cudaGetLastError();
 }

@@ -99,7 +99,22 @@ struct ComposeArgs {
     const void *y1, *y2, *w1, *w2;
     void *out;
     int M, N, K1, K2;
+    int phase;               // MATE_PHASE_* reported for the launch (0: MATE_PHASE_COMPOSE)
     int *err;                // device error word
+};
+
+// MA-branch front-end (mate_frontend_fwd): in_proj, causal conv along the scan
+// order, SiLU, softplus(dt + bias). dc = d_inner + 2 G Ns conv channels.
+struct FrontArgs {
+    const void *u, *w_in;                 // (batch*N, d_model), (d_inner + dc + nh, d_model) bf16
+    const float *conv_w, *conv_b, *dt_bias;  // (dc, 4), (dc), (nh)
+    void *z, *x, *B, *C;                  // outputs, grid order, bf16
+    float *dt;                            // (batch*N, nh) fp32
+    void *xbc_pre, *dt_pre;               // workspace: (batch*N, dc), (batch*N, nh) bf16
+    int batch, T, H, W, N, mode;
+    int d_model, d_inner, nh, G, Ns, dc;
+    FastDiv dT, dH, dW, dHW;
+    int *err;                             // device error word
 };
 
 // Phase hook and launch counter (mate_set_phase_hook / mate_kernel_launches).
@@ -137,6 +152,8 @@ bool tesa_tc_supported(const TesaArgs &a);
 cudaError_t launch_tesa_tc(const TesaArgs &a, cudaStream_t s);
 bool compose_tc_supported(const ComposeArgs &a);
 cudaError_t launch_compose_tc(const ComposeArgs &a, cudaStream_t s);
+bool front_supported(const FrontArgs &a);
+cudaError_t launch_front(const FrontArgs &a, cudaStream_t s);
 // tensor-core bi-SSD path (bf16, head dim 64, d_state 64, both directions)
 bool ssd_tc_supported(const SsdArgs &a);
 cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s);

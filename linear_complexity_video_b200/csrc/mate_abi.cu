@@ -216,6 +216,43 @@ SsdWorkspace ssd_workspace_layout(const SsdArgs &a)
     return l;
 }
 
+// shape checks of the front-end; fills a (pointers left null) and the workspace split
+int front_shape(int T, int H, int W, int scan_mode, const mate_frontend_dims *d, FrontArgs &a, size_t &ws_pre,
+                size_t &ws_total)
+{
+    if (!d || T <= 0 || H <= 0 || W <= 0 || d->batch <= 0 || d->d_model <= 0 || d->nheads <= 0 || d->headdim <= 0 ||
+        d->ngroups <= 0 || d->dstate <= 0)
+        return MATE_ERR_INVALID_ARG;
+    if (scan_mode < 0 || scan_mode > MATE_SCAN_ZZ) return MATE_ERR_INVALID_ARG;
+    const int64_t N = (int64_t)T * H * W;
+    if (N >= ((int64_t)1 << 31) || N * d->batch >= ((int64_t)1 << 31)) return MATE_ERR_INVALID_ARG;
+    if (d->nheads % d->ngroups) return MATE_ERR_INVALID_ARG;
+    if (d->dtype != MATE_BF16) return MATE_ERR_UNSUPPORTED;
+    memset(&a, 0, sizeof(a));
+    a.batch = d->batch;
+    a.T = T;
+    a.H = H;
+    a.W = W;
+    a.N = (int)N;
+    a.mode = scan_mode;
+    a.d_model = d->d_model;
+    a.nh = d->nheads;
+    a.d_inner = d->nheads * d->headdim;
+    a.G = d->ngroups;
+    a.Ns = d->dstate;
+    a.dc = a.d_inner + 2 * a.G * a.Ns;
+    a.dT = make_fastdiv(T);
+    a.dH = make_fastdiv(H);
+    a.dW = make_fastdiv(W);
+    a.dHW = make_fastdiv((uint32_t)(H * W));
+    if (!front_supported(a) || a.nh % 8) return MATE_ERR_UNSUPPORTED;
+    const size_t M = (size_t)a.batch * a.N;
+    ws_pre = align_up(M * a.dc * 2);
+    ws_total = ws_pre + align_up(M * a.nh * 2);
+    return MATE_OK;
+}
+
+
 }  // namespace mate
 
 using namespace mate;
@@ -309,7 +346,7 @@ int mate_compose_fwd(const void *y_ma, const void *y_te, const void *w_ma, const
     a.N = d->d_model;
     a.K1 = d->k_ma;
     a.K2 = d->k_te;
-    if (!compose_tc_supported(a)) return MATE_ERR_UNSUPPORTED;
+    if (a.N % 64 || !compose_tc_supported(a)) return MATE_ERR_UNSUPPORTED;
     if (!out || (a.K1 && (!y_ma || !w_ma)) || (a.K2 && (!y_te || !w_te))) return MATE_ERR_INVALID_ARG;
     const void *ptrs[5] = {y_ma, y_te, w_ma, w_te, out};
     for (const void *p : ptrs)
@@ -326,6 +363,63 @@ int mate_compose_fwd(const void *y_ma, const void *y_te, const void *w_ma, const
     a.err = error_word_ptr();
     if (!a.err) return MATE_ERR_CUDA;
     return launch_compose_tc(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
+
+size_t mate_frontend_workspace_bytes(int T, int H, int W, const mate_frontend_dims *d)
+{
+    FrontArgs a;
+    size_t pre = 0, total = 0;
+    if (front_shape(T, H, W, MATE_SCAN_SR, d, a, pre, total) != MATE_OK) return 0;
+    return total;
+}
+
+int mate_frontend_fwd(const void *u, const void *w_in, const float *conv_w, const float *conv_b, const float *dt_bias,
+                      int T, int H, int W, int scan_mode, void *z, void *x, float *dt, void *B, void *C,
+                      const mate_frontend_dims *d, void *workspace, size_t ws_bytes, void *stream)
+{
+    FrontArgs a;
+    size_t pre = 0, total = 0;
+    int rc = front_shape(T, H, W, scan_mode, d, a, pre, total);
+    if (rc != MATE_OK) return rc;
+    if (!u || !w_in || !conv_w || !conv_b || !dt_bias || !z || !x || !dt || !B || !C) return MATE_ERR_INVALID_ARG;
+    const void *bf[7] = {u, w_in, z, x, B, C, workspace};
+    for (const void *p : bf)
+        if (p && !aligned(p, 16)) return MATE_ERR_INVALID_ARG;
+    if (!aligned(conv_w, 4) || !aligned(conv_b, 4) || !aligned(dt_bias, 4) || !aligned(dt, 4))
+        return MATE_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < total || !aligned(workspace, 256)) return MATE_ERR_WORKSPACE;
+    const size_t M = (size_t)a.batch * a.N;
+    const size_t ub = M * a.d_model * 2, wb = (size_t)(a.d_inner + a.dc + a.nh) * a.d_model * 2;
+    const size_t zb = M * a.d_inner * 2, bb = M * a.G * a.Ns * 2, db = M * a.nh * 4;
+    // every output disjoint from every input, from the workspace and from the other outputs
+    const struct {
+        const void *p;
+        size_t n;
+    } outs[5] = {{z, zb}, {x, zb}, {B, bb}, {C, bb}, {dt, db}},
+      ins[6] = {{u, ub}, {w_in, wb}, {conv_w, (size_t)a.dc * 16}, {conv_b, (size_t)a.dc * 4},
+                {dt_bias, (size_t)a.nh * 4}, {workspace, total}};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 6; ++j)
+            if (overlaps(outs[i].p, outs[i].n, ins[j].p, ins[j].n)) return MATE_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 5; ++j)
+            if (overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return MATE_ERR_INVALID_ARG;
+    }
+    a.u = u;
+    a.w_in = w_in;
+    a.conv_w = conv_w;
+    a.conv_b = conv_b;
+    a.dt_bias = dt_bias;
+    a.z = z;
+    a.x = x;
+    a.B = B;
+    a.C = C;
+    a.dt = dt;
+    a.xbc_pre = workspace;
+    a.dt_pre = static_cast<char *>(workspace) + pre;
+    a.err = error_word_ptr();
+    if (!a.err) return MATE_ERR_CUDA;
+    return launch_front(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
 }
 
 int mate_debug_rms_map(int T, int H, int W, int scan_mode, int flip, int32_t *out_dev, void *stream)

@@ -161,6 +161,61 @@ class Oracle:
         return out.reshape(*lead, N)
 
 
+    # ---- MA-branch front-end ------------------------------------------------
+    def frontend(self, u, w_in, conv_w, conv_b, dt_bias, mode: int, nheads: int, headdim: int, ngroups: int,
+                 dstate: int, positions=None):
+        """The standard Mamba2 input side ([Review] section 三, MA-Branch item 1, bidirectional
+        Mamba2; the pages give no more of the block; reading R8 of the C oracle's header):
+            [z | xBC_pre | dt_raw] = u w_in^T
+            xBC[n] = SiLU(conv_b + sum_{k=0..3} conv_w[:, k] xBC_pre[n - 3 + k])   along the scan
+                     order of `mode` (positions before 0 are zero)
+            dt = softplus(dt_raw + dt_bias)
+        u: (batch, T, H, W, d_model). Returns z, x, dt, B, C in grid order, shaped as the SSD takes
+        them. With `positions` (scan positions), only those tokens are produced, as arrays
+        (batch, len(positions), ...) in the order given: the projection is then taken of those
+        tokens and their three predecessors only."""
+        u, w, cw, cb, db = map(_f64, (u, w_in, conv_w, conv_b, dt_bias))
+        b, T, H, W, dm = u.shape
+        N = T * H * W
+        d_inner, gns = nheads * headdim, ngroups * dstate
+        dc = d_inner + 2 * gns
+        order = self.rms_sequence(T, H, W, mode).astype(np.int64)   # scan position -> grid offset
+        flat = u.reshape(b, N, dm)
+        if positions is None:
+            pos = np.arange(N)
+        else:
+            pos = np.asarray(positions, dtype=np.int64)
+        # the tokens needed: each output position and its three predecessors in scan order
+        need = np.unique(np.concatenate([pos - k for k in range(4)]))
+        need = need[need >= 0]
+        proj = flat[:, order[need], :] @ w.T                  # (b, len(need), d_inner + dc + nheads)
+        at = {int(p): i for i, p in enumerate(need)}
+        def pre(p):  # xBC_pre at scan position p (zero before the sequence)
+            return proj[:, at[p], d_inner:d_inner + dc] if p >= 0 else np.zeros((b, dc))
+        conv = np.empty((b, len(pos), dc))
+        for j, p in enumerate(pos):
+            acc = cb.copy()[None, :].repeat(b, axis=0)
+            for k in range(4):
+                acc = acc + cw[:, k][None, :] * pre(int(p) - 3 + k)
+            conv[:, j] = acc
+        act = conv / (1.0 + np.exp(-conv))                    # SiLU
+        rows = np.array([at[int(p)] for p in pos])
+        z = proj[:, rows, :d_inner]
+        dt = np.logaddexp(0.0, proj[:, rows, d_inner + dc:] + db[None, None, :])  # softplus
+        x, Bm, Cm = act[..., :d_inner], act[..., d_inner:d_inner + gns], act[..., d_inner + gns:]
+        if positions is not None:
+            return (z, x.reshape(b, -1, nheads, headdim), dt, Bm.reshape(b, -1, ngroups, dstate),
+                    Cm.reshape(b, -1, ngroups, dstate))
+        # scatter the scan-ordered results back to grid order
+        def grid(a):
+            g = np.empty_like(a)
+            g[:, order] = a
+            return g
+        shp = (b, T, H, W)
+        return (grid(z).reshape(*shp, d_inner), grid(x).reshape(*shp, nheads, headdim), grid(dt).reshape(*shp, nheads),
+                grid(Bm).reshape(*shp, ngroups, dstate), grid(Cm).reshape(*shp, ngroups, dstate))
+
+
 _default: Optional[Oracle] = None
 
 

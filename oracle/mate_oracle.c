@@ -41,6 +41,10 @@
  *      of oracle_zigzag, used only as the comparison order.
  *   R7 MATE composition: the two branch outputs (different widths) are each
  *      projected to the model width and added; no gate, no bias.
+ *   R8 MA-branch front-end (oracle/__init__.py, Oracle.frontend): the standard
+ *      Mamba2 input side, in_proj to [z | x B C | dt], a causal depthwise
+ *      conv of width 4 with bias along the forward scan order, SiLU, and
+ *      softplus(dt + bias); one result feeds both scan directions.
  */
 #include <math.h>
 #include <stdint.h>

@@ -387,6 +387,52 @@ def pin_compose(o):
     assert not np.allclose(full, y1 @ w1.T + y2 @ (w2[::-1]).T)
 
 
-ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_zigzag, pin_compose, pin_pool, pin_scan_dual,
+def pin_frontend(o):
+    """MA-branch front-end (reading R8). In spatial-row order the scan is the grid order, so
+    each channel's conv is numpy's full convolution with the reversed taps, cut to the
+    sequence (the causal conv); an impulse placed at one scan position of the temporal-column
+    order reaches exactly that position and the next three, in scan order, through the taps
+    w3, w2, w1, w0; z is the plain projection; dt is softplus(dt_raw + bias); the sampled form
+    agrees with the full one."""
+    rng = np.random.default_rng(6)
+    b, T, H, W, dm, nh, P, G, Ns = 2, 2, 3, 4, 16, 2, 4, 1, 4
+    d_inner, dc = nh * P, nh * P + 2 * G * Ns
+    u = rng.standard_normal((b, T, H, W, dm))
+    w_in = rng.standard_normal((d_inner + dc + nh, dm)) / 4
+    cw, cb, db = rng.standard_normal((dc, 4)), rng.standard_normal(dc), rng.standard_normal(nh)
+    z, x, dt, Bm, Cm = o.frontend(u, w_in, cw, cb, db, 0, nh, P, G, Ns)
+    proj = u.reshape(b, -1, dm) @ w_in.T
+    _close(z.reshape(b, -1, d_inner), proj[..., :d_inner], 1e-12, "z is not the projection")
+    _close(dt.reshape(b, -1, nh), np.log1p(np.exp(proj[..., d_inner + dc:] + db)), 1e-12, "dt softplus")
+    N = T * H * W
+    act = np.concatenate([x.reshape(b, N, -1), Bm.reshape(b, N, -1), Cm.reshape(b, N, -1)], axis=-1)
+    for bb in range(b):
+        for c in range(dc):
+            v = np.convolve(proj[bb, :, d_inner + c], cw[c, ::-1])[:N] + cb[c]
+            _close(act[bb, :, c], v / (1 + np.exp(-v)), 1e-12, "causal conv in scan order")
+    # impulse in temporal-column order: u chosen so that xBC_pre is one hot at scan position p
+    T, H, W, dm = 4, 3, 2, 8
+    w_in = np.zeros((d_inner + dc + nh, dm))
+    w_in[d_inner, 0] = 1.0                  # channel 0 of xBC_pre reads u[..., 0]
+    order = o.rms_sequence(T, H, W, 3)
+    p = 5
+    u = np.zeros((1, T, H, W, dm))
+    u.reshape(1, -1, dm)[0, order[p], 0] = 1.0
+    cw, cb = rng.standard_normal((dc, 4)), np.zeros(dc)
+    z, x, dt, Bm, Cm = o.frontend(u, w_in, cw, cb, np.zeros(nh), 3, nh, P, G, Ns)
+    got = x.reshape(1, -1, d_inner)[0, order, 0]    # channel 0 along the scan
+    want = np.zeros(T * H * W)
+    for j in range(4):
+        v = cw[0, 3 - j]
+        want[p + j] = v / (1 + np.exp(-v))
+    _close(got, want, 1e-12, "impulse response along the scan order")
+    # the sampled form gives the same rows
+    pos = [0, 3, 11, 23]
+    zs, xs, dts, Bs, Cs = o.frontend(u, w_in, cw, cb, np.zeros(nh), 3, nh, P, G, Ns, positions=pos)
+    _close(xs.reshape(1, len(pos), -1), x.reshape(1, -1, d_inner)[:, order[pos]], 1e-12, "sampled rows")
+
+
+ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_zigzag, pin_compose, pin_frontend, pin_pool,
+            pin_scan_dual,
             pin_scan_closed_forms, pin_bissd_dual, pin_bissd_flip_equivariance, pin_bissd_review,
             pin_tesa_golden, pin_tesa_tiling, pin_tesa_block_mask, pin_tesa_special]

@@ -56,3 +56,31 @@ def test_mutant_is_caught(tmp_path, name, orig, mutated):
         except (AssertionError, ValueError):
             caught.append(pin.__name__)
     assert caught, f"no pin catches the mutant '{name}'"
+
+
+# The front-end part of the oracle is written with numpy (Oracle.frontend); its
+# mutants patch that method's source and rebind it on an oracle instance.
+PY_MUTANTS = [
+    ("front-end taps reversed", "acc = acc + cw[:, k][None, :] * pre(int(p) - 3 + k)",
+     "acc = acc + cw[:, 3 - k][None, :] * pre(int(p) - 3 + k)"),
+    ("front-end conv in grid order", "order = self.rms_sequence(T, H, W, mode).astype(np.int64)",
+     "order = np.arange(T * H * W)"),
+    ("front-end dt without its bias", "proj[:, rows, d_inner + dc:] + db[None, None, :]", "proj[:, rows, d_inner + dc:]"),
+    ("front-end without SiLU", "act = conv / (1.0 + np.exp(-conv))", "act = conv"),
+]
+
+
+@pytest.mark.parametrize("name,orig,mutated", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_python_mutant_is_caught(name, orig, mutated):
+    import inspect
+    import textwrap
+    import types
+
+    src = inspect.getsource(oracle.Oracle.frontend)
+    assert src.count(orig) == 1, f"mutation anchor not found exactly once: {orig!r}"
+    ns = {}
+    exec(textwrap.dedent(src.replace(orig, mutated)), dict(vars(oracle)), ns)
+    o = oracle.Oracle()
+    o.frontend = types.MethodType(ns["frontend"], o)
+    with pytest.raises((AssertionError, ValueError, KeyError)):
+        oracle_pins.pin_frontend(o)

@@ -118,6 +118,25 @@ def generate_compose(tokens: int, k_ma: int, k_te: int, d_model: int = D_MODEL, 
     return {k: v.to(dtype) for k, v in dict(y_ma=y_ma, y_te=y_te, w_ma=w_ma, w_te=w_te).items()}
 
 
+def generate_frontend(cfg: Config, seed: int = 0, d_model: int = D_MODEL) -> Dict[str, torch.Tensor]:
+    """Inputs of the MA-branch front-end for a grid: the block input u ~ N(0, 1)
+    (batch, T, H, W, d_model) bf16, a random-init in_proj w_in ~ N(0, 1/d_model)
+    (rows z, x, B, C, dt) bf16, conv taps and biases ~ U(-1/2, 1/2) fp32 (the
+    uniform range of a width-4 conv's default init), and dt_bias = -4 fp32, so
+    that dt = softplus(N(0, 1) - 4) as in the SSD inputs above. From a generator
+    seeded with seed + 3 in the order u, w_in, conv_w, conv_b."""
+    g = torch.Generator().manual_seed(seed + 3)
+    d_inner = cfg.nheads * cfg.headdim
+    dc = d_inner + 2 * cfg.ngroups * cfg.dstate
+    u = torch.randn(cfg.batch, cfg.T, cfg.H, cfg.W, d_model, generator=g)
+    w_in = torch.randn(d_inner + dc + cfg.nheads, d_model, generator=g) / math.sqrt(d_model)
+    conv_w = torch.rand(dc, 4, generator=g) - 0.5
+    conv_b = torch.rand(dc, generator=g) - 0.5
+    dt_bias = torch.full((cfg.nheads,), -4.0)
+    return {"u": u.to(torch.bfloat16), "w_in": w_in.to(torch.bfloat16), "conv_w": conv_w.float(),
+            "conv_b": conv_b.float(), "dt_bias": dt_bias}
+
+
 def sweep_configs():
     """N from 8k to 131k tokens at H=W=32 with the 131k grid's other settings."""
     base = CONFIGS[HEADLINE]
