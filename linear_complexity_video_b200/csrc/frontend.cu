@@ -13,8 +13,8 @@
 //
 // Launches: three tensor-core GEMMs (compose_tc.cu, one input part each) for z,
 // the conv channels and dt_raw (bf16, the last two into the workspace), then
-// one kernel for the conv and SiLU over 128 scan positions x 128 channels per
-// CTA (rows staged in shared memory with their 3-position halo), and one for dt.
+// one kernel for the conv and SiLU (each warp 16 scan positions x 64 channels,
+// its 19 input rows loaded at once), and one for dt.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -26,8 +26,6 @@ namespace mate {
 
 namespace {
 
-constexpr int kPos = 128;     // scan positions per CTA
-constexpr int kCh = 128;      // conv channels per CTA
 constexpr int kHalo = 3;      // conv width - 1
 constexpr int kThreads = 256;
 
@@ -63,69 +61,68 @@ __device__ __forceinline__ int front_offset(int n, const FrontArgs &a)
     }
 }
 
-// Conv + SiLU for scan positions [s0, s0 + 128) and channels [c0, c0 + 128) of
-// batch element b. Thread t takes the channel pair (c0 + 2 (t % 64), +1) over the
-// 32 positions 32 (t / 64) .. and slides the width-4 window along them.
+// Conv + SiLU: warp w of a CTA takes the channel pair (64 (8 blockIdx.x + w) + 2 lane,
+// +1) of batch element blockIdx.z over the kWarpPos scan positions kWarpPos
+// blockIdx.y ..: it loads the kWarpPos + 3 rows it needs (the halo included) with
+// all loads in flight at once, then slides the width-4 window along them. For every position a
+// warp reads and writes 128 contiguous bytes of a token row, and the CTA's eight
+// warps cover 1 KB of it.
+constexpr int kWarpPos = 16;
 __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
 {
-    __shared__ __align__(16) __nv_bfloat16 rows[kPos + kHalo][kCh];
-    __shared__ int goff[kPos];
-    const int tid = threadIdx.x;
-    const int s0 = blockIdx.x * kPos, c0 = blockIdx.y * kCh, b = blockIdx.z;
-    const int nch = min(kCh, a.dc - c0);  // channels of this CTA (a multiple of 8)
-    // grid offsets of the 128 output positions
-    for (int i = tid; i < kPos; i += kThreads) goff[i] = s0 + i < a.N ? front_offset(s0 + i, a) : 0;
-    // the 131 input rows (positions s0 - 3 ..), 16 bytes per request, zeros outside the sequence
-    const __nv_bfloat16 *pre = static_cast<const __nv_bfloat16 *>(a.xbc_pre);
-    for (int q = tid; q < (kPos + kHalo) * (kCh / 8); q += kThreads) {
-        const int i = q / (kCh / 8), cc = (q % (kCh / 8)) * 8;
-        const int p = s0 - kHalo + i;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (p >= 0 && p < a.N && cc < nch) {
-            const int g = front_offset(p, a);
-            v = *reinterpret_cast<const uint4 *>(pre + ((size_t)b * a.N + g) * a.dc + c0 + cc);
-        }
-        *reinterpret_cast<uint4 *>(&rows[i][cc]) = v;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cbase = (blockIdx.x * (kThreads / 32) + warp) * 64;
+    const int c = cbase + 2 * lane;
+    const int s0 = blockIdx.y * kWarpPos, b = blockIdx.z;
+    if (cbase >= a.dc) return;  // (a multiple of 8: whole warps past the channels leave)
+    // grid offsets of positions s0 - 3 + i: lane i computes i < 32 (and, were 35 needed,
+    // lanes 0-2 the positions 32..34)
+    const int p_lo = s0 - kHalo + lane, p_hi = s0 - kHalo + 32 + lane;
+    const int off_lo = (p_lo >= 0 && p_lo < a.N) ? front_offset(p_lo, a) : -1;
+    const int off_hi = (lane < kHalo && p_hi < a.N) ? front_offset(p_hi, a) : -1;
+    const bool live = c < a.dc;
+    const __nv_bfloat16 *pre = static_cast<const __nv_bfloat16 *>(a.xbc_pre) + (size_t)b * a.N * a.dc + c;
+    uint32_t in[kWarpPos + kHalo];
+#pragma unroll
+    for (int i = 0; i < kWarpPos + kHalo; ++i) {
+        const int g = __shfl_sync(0xffffffffu, i < 32 ? off_lo : off_hi, i & 31);
+        in[i] = (g >= 0 && live) ? *reinterpret_cast<const uint32_t *>(pre + (size_t)g * a.dc) : 0u;
     }
-    __syncthreads();
-    const int cp = 2 * (tid % 64), pg = tid / 64;
-    if (cp >= nch) return;
-    const int c = c0 + cp;
+    // lanes past the last channel stay in the loop below (its shuffles take the whole
+    // warp) but read channel 0's taps and store nothing
+    const int cl = live ? c : 0;
     float w0[4], w1[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        w0[k] = a.conv_w[(size_t)c * 4 + k];
-        w1[k] = a.conv_w[(size_t)(c + 1) * 4 + k];
+        w0[k] = a.conv_w[(size_t)cl * 4 + k];
+        w1[k] = a.conv_w[(size_t)(cl + 1) * 4 + k];
     }
-    const float b0 = a.conv_b[c], b1 = a.conv_b[c + 1];
+    const float b0 = a.conv_b[cl], b1 = a.conv_b[cl + 1];
     // where this channel pair goes: x, B or C (a pair never straddles two of them)
     const int gns = a.G * a.Ns;
     __nv_bfloat16 *dst;
     int width, cofs;
-    if (c < a.d_inner) {
-        dst = static_cast<__nv_bfloat16 *>(a.x), width = a.d_inner, cofs = c;
-    } else if (c < a.d_inner + gns) {
-        dst = static_cast<__nv_bfloat16 *>(a.B), width = gns, cofs = c - a.d_inner;
+    if (cl < a.d_inner) {
+        dst = static_cast<__nv_bfloat16 *>(a.x), width = a.d_inner, cofs = cl;
+    } else if (cl < a.d_inner + gns) {
+        dst = static_cast<__nv_bfloat16 *>(a.B), width = gns, cofs = cl - a.d_inner;
     } else {
-        dst = static_cast<__nv_bfloat16 *>(a.C), width = gns, cofs = c - a.d_inner - gns;
+        dst = static_cast<__nv_bfloat16 *>(a.C), width = gns, cofs = cl - a.d_inner - gns;
     }
-    // the window: inputs at positions n-3, n-2, n-1 of the first output n = 32 pg
-    float2 in[3];
+    dst += (size_t)b * a.N * width + cofs;
 #pragma unroll
-    for (int k = 0; k < 3; ++k) in[k] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&rows[32 * pg + k][cp]));
-    for (int j = 0; j < 32; ++j) {
-        const int i = 32 * pg + j;  // output position s0 + i sits at row i + 3
-        const float2 cur = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&rows[i + kHalo][cp]));
-        float v0 = b0 + w0[0] * in[0].x + w0[1] * in[1].x + w0[2] * in[2].x + w0[3] * cur.x;
-        float v1 = b1 + w1[0] * in[0].y + w1[1] * in[1].y + w1[2] * in[2].y + w1[3] * cur.y;
-        v0 = v0 / (1.f + __expf(-v0));  // SiLU
-        v1 = v1 / (1.f + __expf(-v1));
-        if (s0 + i < a.N)
-            *reinterpret_cast<__nv_bfloat162 *>(dst + ((size_t)b * a.N + goff[i]) * width + cofs) =
-                __floats2bfloat162_rn(v0, v1);
-        in[0] = in[1];
-        in[1] = in[2];
-        in[2] = cur;
+    for (int j = 0; j < kWarpPos; ++j) {
+        // output position s0 + j: inputs at rows j .. j + 3 of `in`
+        float2 x4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x4[k] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&in[j + k]));
+        float v0 = b0 + w0[0] * x4[0].x + w0[1] * x4[1].x + w0[2] * x4[2].x + w0[3] * x4[3].x;
+        float v1 = b1 + w1[0] * x4[0].y + w1[1] * x4[1].y + w1[2] * x4[2].y + w1[3] * x4[3].y;
+        v0 = __fdividef(v0, 1.f + __expf(-v0));  // SiLU (for v -> -inf the quotient is 0)
+        v1 = __fdividef(v1, 1.f + __expf(-v1));
+        const int g = __shfl_sync(0xffffffffu, (j + kHalo) < 32 ? off_lo : off_hi, (j + kHalo) & 31);
+        if (g >= 0 && live)
+            *reinterpret_cast<__nv_bfloat162 *>(dst + (size_t)g * width) = __floats2bfloat162_rn(v0, v1);
     }
 }
 
@@ -184,7 +181,9 @@ cudaError_t launch_front(const FrontArgs &a, cudaStream_t s)
     }
     {
         Phase ph(MATE_PHASE_FRONT_CONV, s);
-        front_conv_kernel<<<dim3((a.N + kPos - 1) / kPos, (a.dc + kCh - 1) / kCh, a.batch), kThreads, 0, s>>>(a);
+        front_conv_kernel<<<dim3((a.dc + 64 * (kThreads / 32) - 1) / (64 * (kThreads / 32)),
+                                 (a.N + kWarpPos - 1) / kWarpPos, a.batch),
+                            kThreads, 0, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

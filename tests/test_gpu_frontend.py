@@ -42,6 +42,16 @@ def test_frontend_small_matches_oracle(mode):
         assert rel_err(host64(got), want) <= TOL["bf16"], name
 
 
+def test_frontend_ragged_channels():
+    # 544 conv channels (d_state 16): the last warp of a CTA holds channels past the end
+    cfg = workloads.CONFIGS["tiny"].with_(T=2, H=6, W=11, batch=1, nheads=8, headdim=64, dstate=16, ngroups=1)
+    inp, outs = _run(cfg, 1, 128, seed=11)
+    ref = oracle.get().frontend(inp["u"], inp["w_in"], inp["conv_w"], inp["conv_b"], inp["dt_bias"], 1,
+                                cfg.nheads, cfg.headdim, cfg.ngroups, cfg.dstate)
+    for name, got, want in zip("z x dt B C".split(), outs, ref):
+        assert rel_err(host64(got), want) <= TOL["bf16"], name
+
+
 def test_frontend_block_widths():
     # d_model 2560, 80 heads of 64, d_state 64 (10,448 in_proj rows) on a 4x8x8 grid in TC order
     cfg = workloads.CONFIGS["512p-68s"].with_(T=4, H=8, W=8)
