@@ -3,6 +3,7 @@ prefix scan, the bidirectional SSD scan and TESA over one batch of a
 synthetic latent grid.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl mate|reference]
+    python bench.py --report | --component compose|frontend [--config NAME]
 
 Prints one JSON line (rank 0). With N > 1 (torchrun, one rank per GPU; a
 plain `python bench.py --gpus N` starts the N ranks itself) every rank
@@ -751,6 +752,8 @@ def main():
     ap.add_argument("--chunk", type=int, default=0, help="override the scan chunk length (a tiling choice)")
     ap.add_argument("--report", action="store_true",
                     help="time every bf16 grid in each of its scan orders and the N sweep (one JSON line each)")
+    ap.add_argument("--component", choices=["compose", "frontend"],
+                    help="time one component beside the token mix on --config (one JSON line)")
     ap.add_argument("--steps-ref", type=int, default=1)
     ap.add_argument("--warmup-ref", type=int, default=0)
     args = ap.parse_args()
@@ -777,6 +780,10 @@ def main():
         return
     if args.report:
         run_report(args)
+        return
+    if args.component:
+        fn = time_compose if args.component == "compose" else time_frontend
+        print(json.dumps(fn(cfg, args.steps, args.warmup)), flush=True)
         return
 
     dist = None
