@@ -303,7 +303,7 @@ size_t mate_frontend_workspace_bytes(int T, int H, int W, const mate_frontend_di
  * Device pointers; bf16 ones 16-byte aligned, fp32 ones 4-byte aligned;
  * outputs caller-owned and disjoint from the inputs and the workspace.
  * Supported: d_model a multiple of 64, d_inner and ngroups * dstate even,
- * dc and nheads multiples of 8. Returns MATE_OK, MATE_ERR_INVALID_ARG,
+ * dc and nheads multiples of 8, T*H*W * dc < 2^31. Returns MATE_OK, MATE_ERR_INVALID_ARG,
  * MATE_ERR_UNSUPPORTED, MATE_ERR_WORKSPACE or MATE_ERR_CUDA.
  */
 int mate_frontend_fwd(const void *u, const void *w_in, const float *conv_w, const float *conv_b, const float *dt_bias,

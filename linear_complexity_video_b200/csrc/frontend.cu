@@ -17,6 +17,7 @@
 // its 19 input rows loaded at once), and one for dt.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 #include <cuda_bf16.h>
 
@@ -68,6 +69,16 @@ __device__ __forceinline__ int front_offset(int n, const FrontArgs &a)
 // warp reads and writes 128 contiguous bytes of a token row, and the CTA's eight
 // warps cover 1 KB of it.
 constexpr int kWarpPos = 16;
+
+// SiLU(v) = v sigmoid(v) = v (1 + tanh(v / 2)) / 2, with the hardware tanh
+// (tanh.approx.f32, relative error about 2^-11: far below the bf16 rounding of
+// the result).
+__device__ __forceinline__ float silu(float v)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
+    return 0.5f * v * (1.f + t);
+}
 __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -86,7 +97,8 @@ __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
 #pragma unroll
     for (int i = 0; i < kWarpPos + kHalo; ++i) {
         const int g = __shfl_sync(0xffffffffu, i < 32 ? off_lo : off_hi, i & 31);
-        in[i] = (g >= 0 && live) ? *reinterpret_cast<const uint32_t *>(pre + (size_t)g * a.dc) : 0u;
+        // (g * dc < 2^31: a grid holds fewer than 2^31 elements of a channel group)
+        in[i] = (g >= 0 && live) ? *reinterpret_cast<const uint32_t *>(pre + g * a.dc) : 0u;
     }
     // lanes past the last channel stay in the loop below (its shuffles take the whole
     // warp) but read channel 0's taps and store nothing
@@ -110,19 +122,21 @@ __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
         dst = static_cast<__nv_bfloat16 *>(a.C), width = gns, cofs = cl - a.d_inner - gns;
     }
     dst += (size_t)b * a.N * width + cofs;
+    // every input row unpacked once; the two channels' taps as packed fp32 pairs
+    float2 xin[kWarpPos + kHalo];
+#pragma unroll
+    for (int i = 0; i < kWarpPos + kHalo; ++i) xin[i] = tc::unpack_bf16(in[i]);
+    const float2 tap[4] = {make_float2(w0[0], w1[0]), make_float2(w0[1], w1[1]), make_float2(w0[2], w1[2]),
+                           make_float2(w0[3], w1[3])};
 #pragma unroll
     for (int j = 0; j < kWarpPos; ++j) {
-        // output position s0 + j: inputs at rows j .. j + 3 of `in`
-        float2 x4[4];
+        // output position s0 + j: inputs at rows j .. j + 3
+        float2 v = make_float2(b0, b1);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x4[k] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&in[j + k]));
-        float v0 = b0 + w0[0] * x4[0].x + w0[1] * x4[1].x + w0[2] * x4[2].x + w0[3] * x4[3].x;
-        float v1 = b1 + w1[0] * x4[0].y + w1[1] * x4[1].y + w1[2] * x4[2].y + w1[3] * x4[3].y;
-        v0 = __fdividef(v0, 1.f + __expf(-v0));  // SiLU (for v -> -inf the quotient is 0)
-        v1 = __fdividef(v1, 1.f + __expf(-v1));
+        for (int k = 0; k < 4; ++k) v = tc::fma_f32x2(tap[k], xin[j + k], v);
         const int g = __shfl_sync(0xffffffffu, (j + kHalo) < 32 ? off_lo : off_hi, (j + kHalo) & 31);
         if (g >= 0 && live)
-            *reinterpret_cast<__nv_bfloat162 *>(dst + (size_t)g * width) = __floats2bfloat162_rn(v0, v1);
+            *reinterpret_cast<__nv_bfloat162 *>(dst + g * width) = __floats2bfloat162_rn(silu(v.x), silu(v.y));
     }
 }
 

@@ -246,6 +246,8 @@ int front_shape(int T, int H, int W, int scan_mode, const mate_frontend_dims *d,
     a.dW = make_fastdiv(W);
     a.dHW = make_fastdiv((uint32_t)(H * W));
     if (!front_supported(a) || a.nh % 8) return MATE_ERR_UNSUPPORTED;
+    // the conv addresses a token row of a batch element in 32 bits
+    if (N * a.dc >= ((int64_t)1 << 31)) return MATE_ERR_UNSUPPORTED;
     const size_t M = (size_t)a.batch * a.N;
     ws_pre = align_up(M * a.dc * 2);
     ws_total = ws_pre + align_up(M * a.nh * 2);
