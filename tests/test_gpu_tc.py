@@ -98,6 +98,17 @@ def test_ssd_tc_zigzag_odd_rows():
     assert _run_ssd(cfg, inp, 4, (3, 1, 3), 128) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("chunk", [128, 384, 512])
+def test_ssd_tc_many_items_per_cta(chunk):
+    # 32x16x16 grid, 16 heads, batch 2, TC order (TMA row boxes): 352 to 1,024 (head,
+    # chunk) items per batch element, so each persistent chunk_out CTA walks several
+    # with one to four sub-chunks each (its next item's dt and rows requested during the
+    # current one); with 384 the last chunk is a third full; review runs of 8 along t
+    cfg = workloads.CONFIGS["256p-17s"].with_(nheads=16, batch=2)
+    inp = workloads.generate(cfg, seed=13, parts=("ssd",))
+    assert _run_ssd(cfg, inp, 3, (8, 4, 4), chunk, heads=[0, 7, 15]) <= TOL["bf16"]
+
+
 def test_ssd_tc_review_extremes():
     # one review cell per token (2,048 cells: the cell weights do not fit in shared memory
     # and every h_init part spans several tiles) and one cell for the whole grid (three of
