@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
 baseline use this package; the product path never imports it.
 
 The wrapper marshals arrays only: every step of the computation runs in the
-C file. Inputs are upcast to float64 exactly (bf16 and fp32 values are
+C file, except the MA-branch front-end (Oracle.frontend), written with numpy. Inputs are upcast to float64 exactly (bf16 and fp32 values are
 representable in fp64), so the oracle sees the very values the GPU sees.
 """
 from __future__ import annotations
@@ -64,8 +64,10 @@ class Oracle:
         L.oracle_tesa_window_ids.argtypes = [ctypes.c_int] * 5 + [_intp, _i32p]
         L.oracle_tesa.argtypes = [ctypes.c_int] * 6 + [_f64p] * 3 + [ctypes.c_int] * 2 + [_intp, _f64p]
         L.oracle_compose.argtypes = [ctypes.c_int64] + [ctypes.c_int] * 3 + [_f64p] * 5
+        L.oracle_gate_norm.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_double] + [_f64p] * 4
         for f in ("oracle_unroll", "oracle_rms_sequence", "oracle_avg_pool", "oracle_ssd_scan",
-                  "oracle_bissd", "oracle_tesa_window_ids", "oracle_tesa", "oracle_compose"):
+                  "oracle_bissd", "oracle_tesa_window_ids", "oracle_tesa", "oracle_compose",
+                  "oracle_gate_norm"):
             getattr(L, f).restype = ctypes.c_int
 
     # ---- Rotary Major Scan -------------------------------------------------
@@ -160,6 +162,22 @@ class Oracle:
             raise ValueError(f"oracle_compose rc={rc}")
         return out.reshape(*lead, N)
 
+
+    def gate_norm(self, y, z, w, group: int, eps: float) -> np.ndarray:
+        """Gated RMS norm of the MA-branch output (reading R9): v = y SiLU(z), each group of
+        `group` channels divided by sqrt(mean(v^2) + eps), times w. y, z: (..., C); w: (C,).
+        Returns (..., C)."""
+        y, z, w = map(_f64, (y, z, w))
+        lead, C = y.shape[:-1], y.shape[-1]
+        M = int(np.prod(lead)) if lead else 1
+        y = np.ascontiguousarray(y.reshape(M, C))
+        z = np.ascontiguousarray(z.reshape(M, C))
+        out = np.empty((M, C), dtype=np.float64)
+        rc = self.lib.oracle_gate_norm(M, C, group, ctypes.c_double(eps), _ptr(y, _f64p), _ptr(z, _f64p),
+                                       _ptr(np.ascontiguousarray(w), _f64p), _ptr(out, _f64p))
+        if rc:
+            raise ValueError(f"oracle_gate_norm rc={rc}")
+        return out.reshape(*lead, C)
 
     # ---- MA-branch front-end ------------------------------------------------
     def frontend(self, u, w_in, conv_w, conv_b, dt_bias, mode: int, nheads: int, headdim: int, ngroups: int,

@@ -45,6 +45,10 @@
  *      Mamba2 input side, in_proj to [z | x B C | dt], a causal depthwise
  *      conv of width 4 with bias along the forward scan order, SiLU, and
  *      softplus(dt + bias); one result feeds both scan directions.
+ *   R9 MA-branch output side (oracle_gate_norm): the standard Mamba2 gated RMS
+ *      norm, gate first: v = y * SiLU(z), then each group of `group`
+ *      consecutive channels is divided by the root of its mean square plus eps
+ *      and scaled by the per-channel weight. The pages name the block only.
  */
 #include <math.h>
 #include <stdint.h>
@@ -458,6 +462,36 @@ int oracle_compose(int64_t M, int K1, int K2, int N, const double *y1, const dou
             for (int k = 0; k < K1; ++k) s1 += y1[i * K1 + k] * w1[(int64_t)n * K1 + k];
             for (int k = 0; k < K2; ++k) s2 += y2[i * K2 + k] * w2[(int64_t)n * K2 + k];
             out[i * N + n] = s1 + s2;
+        }
+    }
+    return ORACLE_OK;
+}
+
+
+/*
+ * MA-branch output side (paper review "LinGen ...", section 三, MA-Branch item 1:
+ * the branch is a bidirectional Mamba2 block; reading R9): the bi-SSD output y
+ * gated by the front-end's z and normalised, per row i and channel group g,
+ *     v_k     = y_k z_k / (1 + exp(-z_k))                 (y times SiLU(z))
+ *     out_k   = v_k w_k / sqrt(mean_{k in g} v_k^2 + eps)
+ * y, z, out: (M, C) row-major; w: (C); C a multiple of group.
+ */
+int oracle_gate_norm(int64_t M, int C, int group, double eps, const double *y, const double *z, const double *w,
+                     double *out)
+{
+    if (M < 0 || C <= 0 || group <= 0 || C % group || eps < 0.0 || !y || !z || !w || !out) return ORACLE_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < M; ++i) {
+        for (int g0 = 0; g0 < C; g0 += group) {
+            double ss = 0.0;
+            for (int k = g0; k < g0 + group; ++k) {
+                const double zk = z[i * C + k];
+                const double v = y[i * C + k] * zk / (1.0 + exp(-zk));
+                out[i * C + k] = v;
+                ss += v * v;
+            }
+            const double inv = 1.0 / sqrt(ss / group + eps);
+            for (int k = g0; k < g0 + group; ++k) out[i * C + k] = out[i * C + k] * w[k] * inv;
         }
     }
     return ORACLE_OK;

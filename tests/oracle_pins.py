@@ -432,7 +432,38 @@ def pin_frontend(o):
     _close(xs.reshape(1, len(pos), -1), x.reshape(1, -1, d_inner)[:, order[pos]], 1e-12, "sampled rows")
 
 
-ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_zigzag, pin_compose, pin_frontend, pin_pool,
+def pin_gate_norm(o):
+    """MA-branch output side (reading R9). Against torch's float64 rms_norm of y * silu(z)
+    taken group by group (the library special case); a group whose gated values are all
+    one constant c has the closed form c w / sqrt(c^2 + eps); with eps = 0 every group's
+    mean square of out / w is exactly 1; and SiLU written as z (1 + tanh(z / 2)) / 2, not
+    the oracle's form, gives the ratios inside a group."""
+    rng = np.random.default_rng(7)
+    M, C, group, eps = 6, 24, 8, 0.5
+    y, z, w = rng.standard_normal((M, C)), rng.standard_normal((M, C)) * 2, rng.standard_normal(C)
+    got = o.gate_norm(y, z, w, group, eps)
+    yt, zt = torch.from_numpy(y), torch.from_numpy(z)
+    v = (yt * torch.nn.functional.silu(zt)).reshape(M, C // group, group)
+    want = torch.nn.functional.rms_norm(v, (group,), eps=eps).reshape(M, C) * torch.from_numpy(w)
+    _close(got, want.numpy(), 1e-12, "gate norm against torch rms_norm of y silu(z)")
+    # every group's gated values equal to one constant c
+    silu = 0.5 * z * (1.0 + np.tanh(0.5 * z))
+    c = np.repeat(rng.uniform(0.2, 2.0, (M, C // group)), group, axis=1)
+    yc = c / silu
+    _close(o.gate_norm(yc, z, w, group, eps), c * w / np.sqrt(c * c + eps), 1e-10, "constant group closed form")
+    # eps = 0: unit mean square per group, and the in-group ratios of the gated values
+    g0 = o.gate_norm(y, z, w, group, 0.0) / w
+    _close(np.mean(g0.reshape(M, C // group, group) ** 2, axis=-1), np.ones((M, C // group)), 1e-12,
+           "mean square per group")
+    gated = (y * silu).reshape(M, C // group, group)
+    ratio = g0.reshape(M, C // group, group) / gated
+    _close(ratio, np.repeat(ratio[..., :1], group, axis=-1), 1e-10, "one scale per group")
+    # the group size matters
+    assert not np.allclose(o.gate_norm(y, z, w, C, eps), got)
+
+
+ALL_PINS = [pin_rms_golden, pin_rms_flip_golden, pin_rms_properties, pin_zigzag, pin_compose, pin_frontend,
+            pin_gate_norm, pin_pool,
             pin_scan_dual,
             pin_scan_closed_forms, pin_bissd_dual, pin_bissd_flip_equivariance, pin_bissd_review,
             pin_tesa_golden, pin_tesa_tiling, pin_tesa_block_mask, pin_tesa_special]

@@ -33,6 +33,14 @@ MUTANTS = [
     ("composition drops the TE branch", "out[i * N + n] = s1 + s2;", "out[i * N + n] = s1;"),
     ("composition reads w1 transposed", "s1 += y1[i * K1 + k] * w1[(int64_t)n * K1 + k];",
      "s1 += y1[i * K1 + k] * w1[(int64_t)(k % N) * K1 + n % K1];"),
+    ("gate norm without the gate", "const double v = y[i * C + k] * zk / (1.0 + exp(-zk));",
+     "const double v = y[i * C + k];"),
+    ("gate norm with a sigmoid gate", "const double v = y[i * C + k] * zk / (1.0 + exp(-zk));",
+     "const double v = y[i * C + k] / (1.0 + exp(-zk));"),
+    ("gate norm over the sum, not the mean", "1.0 / sqrt(ss / group + eps);", "1.0 / sqrt(ss + eps);"),
+    ("gate norm eps outside the root", "1.0 / sqrt(ss / group + eps);", "1.0 / (sqrt(ss / group) + eps);"),
+    ("gate norm without its weight", "out[i * C + k] = out[i * C + k] * w[k] * inv;",
+     "out[i * C + k] = out[i * C + k] * inv;"),
     ("softmax without 1/sqrt(d)", "const double scale = 1.0 / sqrt((double)d);", "const double scale = 1.0;"),
     ("window boundaries at -shift", "for (int b = s; b < Lx; b += S) starts[n++] = b;",
      "for (int b = (S - s) % S; b < Lx; b += S) starts[n++] = b;"),
