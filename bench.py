@@ -3,7 +3,7 @@ prefix scan, the bidirectional SSD scan and TESA over one batch of a
 synthetic latent grid.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl mate|reference]
-    python bench.py --report | --component compose|frontend [--config NAME]
+    python bench.py --report | --component compose|frontend|gate_norm [--config NAME]
 
 Prints one JSON line (rank 0). With N > 1 (torchrun, one rank per GPU; a
 plain `python bench.py --gpus N` starts the N ranks itself) every rank
@@ -514,6 +514,47 @@ def time_compose(cfg, steps, warmup, sample_rows=32):
             "oracle_s_scaled": round(t_or, 1), "oracle_sample_rows": sample_rows}
 
 
+def time_gate_norm(cfg, steps, warmup, sample_rows=256):
+    """mate_gate_norm_fwd on the grid's bi-SSD output rows (tokens, nh*P), one norm group
+    per row (ngroups = 1): device time from CUDA events, the HBM fraction by its
+    algorithmic bytes (y and z read once, out written once), and the oracle timed on
+    `sample_rows` rows, scaled to all rows."""
+    import torch
+
+    import linear_complexity_video_b200 as mate
+    import oracle
+
+    c = cfg.nheads * cfg.headdim
+    group = c // cfg.ngroups
+    host = workloads.generate_gate_norm(cfg.tokens, c, seed=0)
+    d = {k: v.cuda() for k, v in host.items()}
+    out = torch.empty(cfg.tokens, c, dtype=torch.bfloat16, device="cuda")
+    for _ in range(warmup):
+        mate.gate_norm(d["y"], d["z"], d["w"], group, 1e-5, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        mate.gate_norm(d["y"], d["z"], d["w"], group, 1e-5, out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    if mate.mate_last_error() != 0:
+        raise RuntimeError("device error word set")
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = 3.0 * 2 * cfg.tokens * c + 4.0 * c
+    peaks, _ = load_peaks()
+    t0 = time.perf_counter()
+    oracle.get().gate_norm(host["y"][:sample_rows], host["z"][:sample_rows], host["w"], group, 1e-5)
+    t_or = (time.perf_counter() - t0) * cfg.tokens / sample_rows
+    del d, out
+    torch.cuda.empty_cache()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"report": "gate_norm", "workload": cfg.name, "tokens": cfg.tokens, "channels": c, "group": group,
+            "ms": round(ms, 4), "gbs": round(gbs, 1), "hbm_peak": float(peaks["hbm_gbs"]),
+            "hbm_frac": round(gbs / float(peaks["hbm_gbs"]), 4), "mtokens_per_s": round(cfg.tokens / ms / 1e3, 2),
+            "oracle_s_scaled": round(t_or, 2), "oracle_sample_rows": sample_rows}
+
+
 def time_frontend(cfg, steps, warmup):
     """mate_frontend_fwd on the grid (d_model 2560 to z, x, B, C, dt): device time
     from CUDA events, the split by phase from the phase hook, the in_proj GEMMs
@@ -621,6 +662,7 @@ def run_report(args):
     # the headline grid, against the tensor-core roofline; the oracle on a row sample
     print(json.dumps(time_compose(cfg, args.steps, args.warmup)), flush=True)
     print(json.dumps(time_frontend(cfg, args.steps, args.warmup)), flush=True)
+    print(json.dumps(time_gate_norm(cfg, args.steps, args.warmup)), flush=True)
     Ns, ts = [], []
     for cfg in workloads.sweep_configs():
         ms, phases = time_config(cfg, cfg.modes[0], args.steps, args.warmup)
@@ -756,7 +798,7 @@ def main():
     ap.add_argument("--chunk", type=int, default=0, help="override the scan chunk length (a tiling choice)")
     ap.add_argument("--report", action="store_true",
                     help="time every bf16 grid in each of its scan orders and the N sweep (one JSON line each)")
-    ap.add_argument("--component", choices=["compose", "frontend"],
+    ap.add_argument("--component", choices=["compose", "frontend", "gate_norm"],
                     help="time one component beside the token mix on --config (one JSON line)")
     ap.add_argument("--steps-ref", type=int, default=1)
     ap.add_argument("--warmup-ref", type=int, default=0)
@@ -786,7 +828,7 @@ def main():
         run_report(args)
         return
     if args.component:
-        fn = time_compose if args.component == "compose" else time_frontend
+        fn = {"compose": time_compose, "frontend": time_frontend, "gate_norm": time_gate_norm}[args.component]
         print(json.dumps(fn(cfg, args.steps, args.warmup)), flush=True)
         return
 

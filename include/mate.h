@@ -262,6 +262,36 @@ typedef struct {
 int mate_compose_fwd(const void *y_ma, const void *y_te, const void *w_ma, const void *w_te, void *out,
                      const mate_compose_dims *d, void *stream);
 
+/* ---- MA-branch output side ----------------------------------------------- */
+typedef struct {
+    int tokens;   /* rows */
+    int channels; /* C = d_inner of the bi-SSD (nheads * headdim, e.g. 5120) */
+    int group;    /* channels per norm group (Mamba2: d_inner / ngroups)       */
+    int dtype;    /* MATE_BF16 (the only storage the kernel takes)             */
+} mate_gate_norm_dims;
+
+/*
+ * MA-branch output side (paper review, section 三, MA-Branch item 1, the
+ * bidirectional Mamba2 block; the pages give no more of it, so this is the
+ * standard Mamba2 gated RMS norm, gate first): per row and group of `group`
+ * consecutive channels,
+ *     v_k   = y_k SiLU(z_k)
+ *     out_k = v_k w_k / sqrt(mean_{k in group} v_k^2 + eps)
+ * in fp32, rounded once to bf16. Its output is the MA-branch's input to
+ * mate_compose_fwd.
+ *   y   : (tokens, channels) bf16, row-major (the bi-SSD output viewed as rows)
+ *   z   : (tokens, channels) bf16, row-major (mate_frontend_fwd's z)
+ *   w   : (channels)         fp32, the norm weight
+ *   out : (tokens, channels) bf16, row-major, caller-owned, must not overlap
+ *         y, z or w
+ * All pointers device memory, 16-byte aligned; eps >= 0 and finite. group a
+ * multiple of 8 that divides channels, channels <= 8192, tokens > 0.
+ * Returns MATE_OK, MATE_ERR_INVALID_ARG (bad pointers, sizes, eps or overlap),
+ * MATE_ERR_UNSUPPORTED (other dtype or sizes) or MATE_ERR_CUDA.
+ */
+int mate_gate_norm_fwd(const void *y, const void *z, const float *w, float eps, void *out,
+                       const mate_gate_norm_dims *d, void *stream);
+
 /* ---- MA-branch front-end ------------------------------------------------- */
 typedef struct {
     int batch;
@@ -360,6 +390,7 @@ int mate_last_error(void *stream);
 #define MATE_PHASE_FRONT_PROJ 8  /* mate_frontend_fwd: one in_proj GEMM (3 per call) */
 #define MATE_PHASE_FRONT_CONV 9  /* mate_frontend_fwd: conv along the scan + SiLU   */
 #define MATE_PHASE_FRONT_DT 10   /* mate_frontend_fwd: softplus(dt + bias)          */
+#define MATE_PHASE_GATE_NORM 11  /* mate_gate_norm_fwd                              */
 
 /*
  * Optional enqueue-time hook, for timing phases with events on the caller's

@@ -40,12 +40,13 @@ EXPORTS = (
     "mate_compose_fwd",
     "mate_frontend_workspace_bytes",
     "mate_frontend_fwd",
+    "mate_gate_norm_fwd",
 )
 
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 PHASES = {1: "review_pool", 2: "review_scan", 3: "chunk_state", 4: "state_pass", 5: "chunk_out", 6: "tesa",
-          7: "compose", 8: "front_proj", 9: "front_conv", 10: "front_dt"}
+          7: "compose", 8: "front_proj", 9: "front_conv", 10: "front_dt", 11: "gate_norm"}
 PHASE_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
 
 
@@ -63,6 +64,10 @@ class mate_attn_dims(ctypes.Structure):
 class mate_compose_dims(ctypes.Structure):
     _fields_ = [("tokens", ctypes.c_int), ("k_ma", ctypes.c_int), ("k_te", ctypes.c_int), ("d_model", ctypes.c_int),
                 ("dtype", ctypes.c_int)]
+
+
+class mate_gate_norm_dims(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_int), ("channels", ctypes.c_int), ("group", ctypes.c_int), ("dtype", ctypes.c_int)]
 
 
 class mate_frontend_dims(ctypes.Structure):
@@ -108,6 +113,8 @@ def load() -> ctypes.CDLL:
     L.mate_debug_fastdiv.restype = ctypes.c_int
     L.mate_compose_fwd.argtypes = [_vp] * 5 + [ctypes.POINTER(mate_compose_dims), _vp]
     L.mate_compose_fwd.restype = ctypes.c_int
+    L.mate_gate_norm_fwd.argtypes = [_vp] * 3 + [ctypes.c_float, _vp, ctypes.POINTER(mate_gate_norm_dims), _vp]
+    L.mate_gate_norm_fwd.restype = ctypes.c_int
     L.mate_frontend_workspace_bytes.argtypes = [ctypes.c_int] * 3 + [ctypes.POINTER(mate_frontend_dims)]
     L.mate_frontend_workspace_bytes.restype = ctypes.c_size_t
     L.mate_frontend_fwd.argtypes = [_vp] * 5 + [ctypes.c_int] * 4 + [_vp] * 5 + [ctypes.POINTER(mate_frontend_dims),

@@ -15,7 +15,7 @@ import torch
 
 from . import _lib
 from ._lib import (MATE_BF16, MATE_DIR_BI, MATE_F32, check, mate_attn_dims, mate_compose_dims, mate_frontend_dims,
-                   mate_ssd_dims)
+                   mate_gate_norm_dims, mate_ssd_dims)
 
 _DT = {torch.float32: MATE_F32, torch.bfloat16: MATE_BF16}
 
@@ -91,6 +91,12 @@ def mate_compose_fwd(y_ma, y_te, w_ma, w_te, out, dims: mate_compose_dims, strea
     rc = _lib.load().mate_compose_fwd(_ptr(y_ma), _ptr(y_te), _ptr(w_ma), _ptr(w_te), _ptr(out), ctypes.byref(dims),
                                       _stream_handle(stream))
     check("mate_compose_fwd", rc)
+
+
+def mate_gate_norm_fwd(y, z, w, eps: float, out, dims: mate_gate_norm_dims, stream=None) -> None:
+    rc = _lib.load().mate_gate_norm_fwd(_ptr(y), _ptr(z), _ptr(w), float(eps), _ptr(out), ctypes.byref(dims),
+                                        _stream_handle(stream))
+    check("mate_gate_norm_fwd", rc)
 
 
 def mate_debug_rms_map(T, H, W, scan_mode, flip, out, stream=None) -> None:
@@ -172,6 +178,25 @@ def compose(y_ma, y_te, w_ma, w_te, out: Optional[torch.Tensor] = None, stream=N
         out = torch.empty(*lead, N, dtype=torch.bfloat16, device=y_ma.device)
     dims = mate_compose_dims(M, int(y_ma.shape[-1]), int(y_te.shape[-1]), N, MATE_BF16)
     mate_compose_fwd(y_ma, y_te, w_ma, w_te, out, dims, stream)
+    return out
+
+
+def gate_norm(y, z, w, group: int, eps: float = 1e-5, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """MA-branch output side: out = y SiLU(z) / sqrt(mean over each group of `group` channels
+    of (y SiLU(z))^2 + eps) * w (bf16). y: (..., C), the bi-SSD output with its heads flattened;
+    z: (..., C), the front-end's z; w: (C,) fp32. Returns (..., C)."""
+    _require(y, "y", torch.bfloat16)
+    _require(z, "z", torch.bfloat16)
+    _require(w, "w", torch.float32)
+    if z.shape != y.shape or w.shape != (y.shape[-1],):
+        raise ValueError("y and z must have one shape and w one entry per channel")
+    M = 1
+    for s in y.shape[:-1]:
+        M *= int(s)
+    if out is None:
+        out = torch.empty_like(y)
+    dims = mate_gate_norm_dims(M, int(y.shape[-1]), int(group), MATE_BF16)
+    mate_gate_norm_fwd(y, z, w, eps, out, dims, stream)
     return out
 
 

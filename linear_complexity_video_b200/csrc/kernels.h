@@ -117,6 +117,16 @@ struct FrontArgs {
     int *err;                             // device error word
 };
 
+// MA-branch output side (mate_gate_norm_fwd): out = y SiLU(z) / rms over each
+// group of channels, times w. y, z, out: (M, C) bf16 row-major; w: (C) fp32.
+struct GateNormArgs {
+    const void *y, *z;
+    const float *w;
+    void *out;
+    int M, C, group;
+    float eps;
+};
+
 // Phase hook and launch counter (mate_set_phase_hook / mate_kernel_launches).
 void phase_mark(int phase, int is_end, cudaStream_t s);
 void count_launch();
@@ -154,6 +164,8 @@ bool compose_tc_supported(const ComposeArgs &a);
 cudaError_t launch_compose_tc(const ComposeArgs &a, cudaStream_t s);
 bool front_supported(const FrontArgs &a);
 cudaError_t launch_front(const FrontArgs &a, cudaStream_t s);
+bool gate_norm_supported(const GateNormArgs &a);
+cudaError_t launch_gate_norm(const GateNormArgs &a, cudaStream_t s);
 // tensor-core bi-SSD path (bf16, head dim 64, d_state 64, both directions)
 bool ssd_tc_supported(const SsdArgs &a);
 cudaError_t launch_ssd_tc(const SsdArgs &a, cudaStream_t s);

@@ -368,6 +368,33 @@ int mate_compose_fwd(const void *y_ma, const void *y_te, const void *w_ma, const
 }
 
 
+int mate_gate_norm_fwd(const void *y, const void *z, const float *w, float eps, void *out,
+                       const mate_gate_norm_dims *d, void *stream)
+{
+    if (!d) return MATE_ERR_INVALID_ARG;
+    if (d->tokens <= 0 || d->channels <= 0 || d->group <= 0 || !(eps >= 0.f) || !isfinite(eps))
+        return MATE_ERR_INVALID_ARG;
+    if (d->dtype != MATE_BF16) return MATE_ERR_UNSUPPORTED;
+    GateNormArgs a;
+    a.M = d->tokens;
+    a.C = d->channels;
+    a.group = d->group;
+    a.eps = eps;
+    if (!gate_norm_supported(a)) return MATE_ERR_UNSUPPORTED;
+    if (!y || !z || !w || !out) return MATE_ERR_INVALID_ARG;
+    const void *ptrs[4] = {y, z, w, out};
+    for (const void *p : ptrs)
+        if (!aligned(p, 16)) return MATE_ERR_INVALID_ARG;
+    const size_t rb = (size_t)a.M * a.C * 2;
+    if (overlaps(out, rb, y, rb) || overlaps(out, rb, z, rb) || overlaps(out, rb, w, (size_t)a.C * 4))
+        return MATE_ERR_INVALID_ARG;
+    a.y = y;
+    a.z = z;
+    a.w = w;
+    a.out = out;
+    return launch_gate_norm(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MATE_OK : MATE_ERR_CUDA;
+}
+
 size_t mate_frontend_workspace_bytes(int T, int H, int W, const mate_frontend_dims *d)
 {
     FrontArgs a;

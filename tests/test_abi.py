@@ -223,3 +223,31 @@ def test_compose_rejects_bad_arguments():
     one = _lib.mate_compose_dims(128, 0, 2560, 2560, _lib.MATE_BF16)
     r = ctypes.c_void_p(1 << 40)
     assert L.mate_compose_fwd(None, p, None, r, None, ctypes.byref(one), None) == _lib.MATE_ERR_INVALID_ARG
+
+
+def test_gate_norm_rejects_bad_arguments():
+    """mate_gate_norm_fwd checks its sizes, eps, dtype, pointers and overlaps before any CUDA call."""
+    L = mate.load()
+    base = 1 << 40
+    y, z, w, o = (ctypes.c_void_p(base + i * (1 << 32)) for i in range(4))
+    ok = _lib.mate_gate_norm_dims(128, 5120, 5120, _lib.MATE_BF16)
+    f = ctypes.c_float
+    assert L.mate_gate_norm_fwd(y, z, w, f(1e-5), o, None, None) == _lib.MATE_ERR_INVALID_ARG
+    for bad in [(0, 64, 64), (128, 0, 64), (128, 64, 0), (-1, 64, 64)]:
+        d = _lib.mate_gate_norm_dims(*bad, _lib.MATE_BF16)
+        assert L.mate_gate_norm_fwd(y, z, w, f(1e-5), o, ctypes.byref(d), None) == _lib.MATE_ERR_INVALID_ARG, bad
+    # group not dividing the row, not a multiple of 8, or a row beyond 8192 channels
+    for bad in [(128, 5120, 3000), (128, 120, 12), (128, 16384, 16384)]:
+        d = _lib.mate_gate_norm_dims(*bad, _lib.MATE_BF16)
+        assert L.mate_gate_norm_fwd(y, z, w, f(1e-5), o, ctypes.byref(d), None) == _lib.MATE_ERR_UNSUPPORTED, bad
+    d = _lib.mate_gate_norm_dims(128, 5120, 5120, _lib.MATE_F32)
+    assert L.mate_gate_norm_fwd(y, z, w, f(1e-5), o, ctypes.byref(d), None) == _lib.MATE_ERR_UNSUPPORTED
+    for eps in (-1.0, float("nan"), float("inf")):
+        assert L.mate_gate_norm_fwd(y, z, w, f(eps), o, ctypes.byref(ok), None) == _lib.MATE_ERR_INVALID_ARG, eps
+    assert L.mate_gate_norm_fwd(y, z, None, f(1e-5), o, ctypes.byref(ok), None) == _lib.MATE_ERR_INVALID_ARG
+    assert L.mate_gate_norm_fwd(y, z, w, f(1e-5), ctypes.c_void_p(base + 8), ctypes.byref(ok), None) == \
+        _lib.MATE_ERR_INVALID_ARG  # misaligned
+    # out overlapping y (one row past its start) or w
+    assert L.mate_gate_norm_fwd(y, z, w, f(1e-5), ctypes.c_void_p(base + 5120 * 2), ctypes.byref(ok), None) == \
+        _lib.MATE_ERR_INVALID_ARG
+    assert L.mate_gate_norm_fwd(y, z, o, f(1e-5), o, ctypes.byref(ok), None) == _lib.MATE_ERR_INVALID_ARG

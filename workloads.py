@@ -118,6 +118,18 @@ def generate_compose(tokens: int, k_ma: int, k_te: int, d_model: int = D_MODEL, 
     return {k: v.to(dtype) for k, v in dict(y_ma=y_ma, y_te=y_te, w_ma=w_ma, w_te=w_te).items()}
 
 
+def generate_gate_norm(tokens: int, channels: int, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """Inputs of the MA-branch output side on the host: the bi-SSD output y ~ N(0, 1) and the
+    front-end's z ~ N(0, 1) as (tokens, channels) bf16 rows, and the norm weight
+    w ~ 1 + N(0, 1) / 10 fp32 (an RMS norm weight starts at one), from a generator seeded with
+    seed + 4 in the order y, z, w."""
+    g = torch.Generator().manual_seed(seed + 4)
+    y = torch.randn(tokens, channels, generator=g).to(torch.bfloat16)
+    z = torch.randn(tokens, channels, generator=g).to(torch.bfloat16)
+    w = 1.0 + torch.randn(channels, generator=g) / 10
+    return {"y": y, "z": z, "w": w.float()}
+
+
 def generate_frontend(cfg: Config, seed: int = 0, d_model: int = D_MODEL) -> Dict[str, torch.Tensor]:
     """Inputs of the MA-branch front-end for a grid: the block input u ~ N(0, 1)
     (batch, T, H, W, d_model) bf16, a random-init in_proj w_in ~ N(0, 1/d_model)
