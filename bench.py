@@ -3,7 +3,7 @@ prefix scan, the bidirectional SSD scan and TESA over one batch of a
 synthetic latent grid.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl mate|reference]
-    python bench.py --report | --component compose|frontend|gate_norm [--config NAME]
+    python bench.py --report | --component compose|frontend|gate_norm|block [--config NAME]
 
 Prints one JSON line (rank 0). With N > 1 (torchrun, one rank per GPU; a
 plain `python bench.py --gpus N` starts the N ranks itself) every rank
@@ -555,6 +555,83 @@ def time_gate_norm(cfg, steps, warmup, sample_rows=256):
             "oracle_s_scaled": round(t_or, 2), "oracle_sample_rows": sample_rows}
 
 
+def time_block(cfg, steps, warmup):
+    """One MATE token mixer (api.block: front-end, bi-SSD, gated norm, TE-branch q/k/v
+    projections, TESA, composition) on the grid with model width 2560: device time from
+    CUDA events, the split by phase from the phase hook (the mean over several hooked
+    calls), and the dense GEMMs' rate (in_proj, q/k/v, composition) against the burst
+    bf16 peak."""
+    import torch
+
+    import linear_complexity_video_b200 as mate
+    from linear_complexity_video_b200 import _lib
+
+    host = workloads.generate_block(cfg, seed=0)
+    d = {k: v.cuda() for k, v in host.items()}
+    spec = dict(scan_mode=cfg.modes[0], review_pool=cfg.review, chunk=cfg.chunk, nheads=cfg.nheads,
+                headdim=cfg.headdim, ngroups=cfg.ngroups, dstate=cfg.dstate, attn_heads=cfg.attn_heads,
+                attn_dim=cfg.attn_dim, Tw=cfg.Tw, Sw=cfg.Sw, shift=cfg.shift)
+
+    def call():
+        return mate.block(d["u"], d, **spec)
+
+    for _ in range(warmup):
+        out = call()
+    torch.cuda.synchronize()
+    uuid = str(torch.cuda.get_device_properties(0).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        out = call()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / steps
+    marks, stream = [], torch.cuda.current_stream()
+
+    def hook(ph, is_end, strm, user):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        marks.append((ph, is_end, ev))
+
+    hooked = max(3, steps // 2)
+    L = mate.load()
+    h = _lib.PHASE_HOOK(hook)
+    L.mate_set_phase_hook(h, None)
+    for _ in range(hooked):
+        out = call()
+    torch.cuda.synchronize()
+    L.mate_set_phase_hook(_lib.PHASE_HOOK(), None)
+    if mate.mate_last_error() != 0:
+        raise RuntimeError("device error word set")
+    phases, opened = {}, {}
+    for ph, is_end, ev in marks:
+        if not is_end:
+            opened[ph] = ev
+        else:
+            name = _lib.PHASES[ph]
+            phases[name] = phases.get(name, 0.0) + opened.pop(ph).elapsed_time(ev) / hooked
+    dm = workloads.D_MODEL
+    d_inner, te = cfg.nheads * cfg.headdim, cfg.attn_heads * cfg.attn_dim
+    dc = d_inner + 2 * cfg.ngroups * cfg.dstate
+    gemm = 2.0 * cfg.tokens * dm * ((d_inner + dc + cfg.nheads) + 3 * te + (d_inner + te))
+    gemm_ms = phases.get("front_proj", 0.0) + phases.get("compose", 0.0)
+    peaks, _ = load_peaks()
+    del d, out
+    torch.cuda.empty_cache()
+    return {"report": "block", "workload": cfg.name, "scan": workloads.MODE_NAMES[cfg.modes[0]], "tokens": cfg.tokens,
+            "d_model": dm, "ms": round(ms, 4), "mtokens_per_s": round(cfg.tokens / ms / 1e3, 2),
+            "phase_ms": {k: round(v, 4) for k, v in phases.items()},
+            "gemm_tflop": round(gemm / 1e12, 3),
+            "gemm_tflops": round(gemm / (gemm_ms / 1e3) / 1e12, 1) if gemm_ms else None,
+            "gemm_tensor_frac": round(gemm / (gemm_ms / 1e3) / 1e12 / float(peaks["bf16_tflops"]), 4) if gemm_ms else None,
+            "gemm_tensor_frac_sustained": round(gemm / (gemm_ms / 1e3) / 1e12 / float(peaks["bf16_tflops_sustained"]), 4)
+            if gemm_ms else None, "clocks": clocks}
+
+
 def time_frontend(cfg, steps, warmup):
     """mate_frontend_fwd on the grid (d_model 2560 to z, x, B, C, dt): device time
     from CUDA events, the split by phase from the phase hook, the in_proj GEMMs
@@ -663,6 +740,7 @@ def run_report(args):
     print(json.dumps(time_compose(cfg, args.steps, args.warmup)), flush=True)
     print(json.dumps(time_frontend(cfg, args.steps, args.warmup)), flush=True)
     print(json.dumps(time_gate_norm(cfg, args.steps, args.warmup)), flush=True)
+    print(json.dumps(time_block(cfg, args.steps, args.warmup)), flush=True)
     Ns, ts = [], []
     for cfg in workloads.sweep_configs():
         ms, phases = time_config(cfg, cfg.modes[0], args.steps, args.warmup)
@@ -798,7 +876,7 @@ def main():
     ap.add_argument("--chunk", type=int, default=0, help="override the scan chunk length (a tiling choice)")
     ap.add_argument("--report", action="store_true",
                     help="time every bf16 grid in each of its scan orders and the N sweep (one JSON line each)")
-    ap.add_argument("--component", choices=["compose", "frontend", "gate_norm"],
+    ap.add_argument("--component", choices=["compose", "frontend", "gate_norm", "block"],
                     help="time one component beside the token mix on --config (one JSON line)")
     ap.add_argument("--steps-ref", type=int, default=1)
     ap.add_argument("--warmup-ref", type=int, default=0)
@@ -828,7 +906,8 @@ def main():
         run_report(args)
         return
     if args.component:
-        fn = {"compose": time_compose, "frontend": time_frontend, "gate_norm": time_gate_norm}[args.component]
+        fn = {"compose": time_compose, "frontend": time_frontend, "gate_norm": time_gate_norm,
+              "block": time_block}[args.component]
         print(json.dumps(fn(cfg, args.steps, args.warmup)), flush=True)
         return
 

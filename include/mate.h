@@ -326,7 +326,7 @@ size_t mate_frontend_workspace_bytes(int T, int H, int W, const mate_frontend_di
  *   w_in   : (d_inner + dc + nheads, d_model)       bf16 (nn.Linear layout,
  *            rows z, then x, B, C, then dt)
  *   conv_w : (dc, 4) fp32;  conv_b : (dc) fp32;  dt_bias : (nheads) fp32
- *   z      : (batch, T, H, W, d_inner)              bf16 (the gate, for later)
+ *   z      : (batch, T, H, W, d_inner)              bf16 (the gate of mate_gate_norm_fwd)
  *   x      : (batch, T, H, W, nheads, headdim)      bf16
  *   dt     : (batch, T, H, W, nheads)               fp32
  *   B, C   : (batch, T, H, W, ngroups, dstate)      bf16

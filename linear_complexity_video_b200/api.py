@@ -200,6 +200,47 @@ def gate_norm(y, z, w, group: int, eps: float = 1e-5, out: Optional[torch.Tensor
     return out
 
 
+def linear(x, w, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """x w^T on the tensor cores (bf16): the composition GEMM with one input part.
+    x: (..., K); w: (N, K) in the nn.Linear layout. Returns (..., N)."""
+    _require(x, "x", torch.bfloat16)
+    _require(w, "w", torch.bfloat16)
+    M = 1
+    for s in x.shape[:-1]:
+        M *= int(s)
+    N = int(w.shape[0])
+    if out is None:
+        out = torch.empty(*x.shape[:-1], N, dtype=torch.bfloat16, device=x.device)
+    mate_compose_fwd(x, None, w, None, out, mate_compose_dims(M, int(x.shape[-1]), 0, N, MATE_BF16), stream)
+    return out
+
+
+def block(u, weights, *, scan_mode: int, review_pool, chunk: int, nheads: int, headdim: int, ngroups: int,
+          dstate: int, attn_heads: int, attn_dim: int, Tw: int, Sw: int, shift, eps: float = 1e-5, stream=None,
+          keep: bool = False):
+    """One MATE token mixer, every step in the library's kernels. u: (batch, T, H, W, d_model) bf16.
+        MA-branch: z, x, dt, B, C = front-end(u); y = bi-SSD(x, dt, A, B, C, D) in the RMS order
+                   `scan_mode` with review tokens; y_ma = gated norm(y, z)
+        TE-branch: q, k, v = u w_q^T, u w_k^T, u w_v^T; y_te = TESA(q, k, v)
+        out = y_ma w_ma^T + y_te w_te^T
+    weights: w_in, conv_w, conv_b, dt_bias, A, D, norm_w, w_q, w_k, w_v, w_ma, w_te (as
+    workloads.generate_block draws them). Returns out (batch, T, H, W, d_model), and with
+    `keep` also a dict of the intermediate tensors."""
+    w = weights
+    b, T, H, W, _ = u.shape
+    z, x, dt, B, C = frontend(u, w["w_in"], w["conv_w"], w["conv_b"], w["dt_bias"], scan_mode, nheads, headdim,
+                              ngroups, dstate, stream=stream)
+    y = bissd(x, dt, w["A"], B, C, w["D"], scan_mode, review_pool, chunk=chunk, stream=stream)
+    d_inner = nheads * headdim
+    y_ma = gate_norm(y.view(b, T, H, W, d_inner), z, w["norm_w"], d_inner // ngroups, eps, stream=stream)
+    q, k, v = (linear(u, w[n], stream=stream).view(b, T, H, W, attn_heads, attn_dim) for n in ("w_q", "w_k", "w_v"))
+    y_te = tesa(q, k, v, Tw, Sw, shift, stream=stream)
+    out = compose(y_ma, y_te.view(b, T, H, W, attn_heads * attn_dim), w["w_ma"], w["w_te"], stream=stream)
+    if keep:
+        return out, dict(z=z, x=x, dt=dt, B=B, C=C, y=y, y_ma=y_ma, q=q, k=k, v=v, y_te=y_te)
+    return out
+
+
 def mate_frontend_workspace_bytes(T: int, H: int, W: int, dims: mate_frontend_dims) -> int:
     return int(_lib.load().mate_frontend_workspace_bytes(T, H, W, ctypes.byref(dims)))
 

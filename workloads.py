@@ -149,6 +149,27 @@ def generate_frontend(cfg: Config, seed: int = 0, d_model: int = D_MODEL) -> Dic
             "conv_b": conv_b.float(), "dt_bias": dt_bias}
 
 
+def generate_block(cfg: Config, seed: int = 0, d_model: int = D_MODEL) -> Dict[str, torch.Tensor]:
+    """Input and random-init weights of one MATE token mixer on the host: the front-end's
+    (generate_frontend: u, w_in, conv_w, conv_b, dt_bias), then, from a generator seeded
+    with seed + 5 in this order, the SSD's A = -exp(U(0, ln 16)) and D ~ N(0, 1) (as in
+    generate), the gated norm's weight 1 + N(0, 1) / 10, the TE-branch projections
+    w_q, w_k, w_v ~ N(0, 1 / d_model) and the composition's w_ma, w_te ~ N(0, 1 / (k_ma + k_te))."""
+    out = generate_frontend(cfg, seed=seed, d_model=d_model)
+    g = torch.Generator().manual_seed(seed + 5)
+    d_inner, te = cfg.nheads * cfg.headdim, cfg.attn_heads * cfg.attn_dim
+    A = -torch.exp(torch.rand(cfg.nheads, generator=g) * math.log(16.0))
+    D = torch.randn(cfg.nheads, generator=g)
+    norm_w = 1.0 + torch.randn(d_inner, generator=g) / 10
+    wq, wk, wv = (torch.randn(te, d_model, generator=g) / math.sqrt(d_model) for _ in range(3))
+    scale = 1.0 / math.sqrt(d_inner + te)
+    w_ma = torch.randn(d_model, d_inner, generator=g) * scale
+    w_te = torch.randn(d_model, te, generator=g) * scale
+    out.update(A=A.float(), D=D.float(), norm_w=norm_w.float(), w_q=wq.to(torch.bfloat16), w_k=wk.to(torch.bfloat16),
+               w_v=wv.to(torch.bfloat16), w_ma=w_ma.to(torch.bfloat16), w_te=w_te.to(torch.bfloat16))
+    return out
+
+
 def sweep_configs():
     """N from 8k to 131k tokens at H=W=32 with the 131k grid's other settings."""
     base = CONFIGS[HEADLINE]
