@@ -70,15 +70,18 @@ __device__ __forceinline__ int front_offset(int n, const FrontArgs &a)
 // warps cover 1 KB of it.
 constexpr int kWarpPos = 16;
 
-// SiLU(v) = v sigmoid(v) = v (1 + tanh(v / 2)) / 2, with the hardware tanh
-// (tanh.approx.f32, relative error about 2^-11: far below the bf16 rounding of
-// the result).
-__device__ __forceinline__ float silu(float v)
+// SiLU of a pair, v (1 + tanh(v / 2)) / 2 with the hardware tanh (tanh.approx.f32,
+// relative error about 2^-11: far below the bf16 rounding of the result)
+__device__ __forceinline__ float2 silu2(float2 v)
 {
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
-    return 0.5f * v * (1.f + t);
+    const float2 h = tc::mul_f32x2(v, make_float2(0.5f, 0.5f));
+    float tx, ty;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(tx) : "f"(h.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(ty) : "f"(h.y));
+    return tc::fma_f32x2(h, make_float2(tx, ty), h);
 }
+static_assert(kWarpPos + kHalo <= 32, "one lane per input row");
+
 __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -86,30 +89,28 @@ __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
     const int c = cbase + 2 * lane;
     const int s0 = blockIdx.y * kWarpPos, b = blockIdx.z;
     if (cbase >= a.dc) return;  // (a multiple of 8: whole warps past the channels leave)
-    // grid offsets of positions s0 - 3 + i: lane i computes i < 32 (and, were 35 needed,
-    // lanes 0-2 the positions 32..34)
-    const int p_lo = s0 - kHalo + lane, p_hi = s0 - kHalo + 32 + lane;
-    const int off_lo = (p_lo >= 0 && p_lo < a.N) ? front_offset(p_lo, a) : -1;
-    const int off_hi = (lane < kHalo && p_hi < a.N) ? front_offset(p_hi, a) : -1;
+    // lane i < 19 owns scan position s0 - 3 + i: its grid offset g (-1 outside the
+    // sequence) and the element offset g * dc of its row of conv channels
+    const int p = s0 - kHalo + lane;
+    const int g_own = (lane < kWarpPos + kHalo && p >= 0 && p < a.N) ? front_offset(p, a) : -1;
+    // (g * dc < 2^31: a grid holds fewer than 2^31 elements of a channel group)
+    const int e_own = g_own >= 0 ? g_own * a.dc : -1;
     const bool live = c < a.dc;
-    const __nv_bfloat16 *pre = static_cast<const __nv_bfloat16 *>(a.xbc_pre) + (size_t)b * a.N * a.dc + c;
+    const uint32_t *pre =
+        reinterpret_cast<const uint32_t *>(static_cast<const __nv_bfloat16 *>(a.xbc_pre) + (size_t)b * a.N * a.dc + c);
     uint32_t in[kWarpPos + kHalo];
 #pragma unroll
     for (int i = 0; i < kWarpPos + kHalo; ++i) {
-        const int g = __shfl_sync(0xffffffffu, i < 32 ? off_lo : off_hi, i & 31);
-        // (g * dc < 2^31: a grid holds fewer than 2^31 elements of a channel group)
-        in[i] = (g >= 0 && live) ? *reinterpret_cast<const uint32_t *>(pre + g * a.dc) : 0u;
+        const int e = __shfl_sync(0xffffffffu, e_own, i);
+        in[i] = (e >= 0 && live) ? pre[e >> 1] : 0u;  // (e and c even: a whole bf16 pair)
     }
     // lanes past the last channel stay in the loop below (its shuffles take the whole
     // warp) but read channel 0's taps and store nothing
     const int cl = live ? c : 0;
-    float w0[4], w1[4];
+    float2 tap[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        w0[k] = a.conv_w[(size_t)cl * 4 + k];
-        w1[k] = a.conv_w[(size_t)(cl + 1) * 4 + k];
-    }
-    const float b0 = a.conv_b[cl], b1 = a.conv_b[cl + 1];
+    for (int k = 0; k < 4; ++k) tap[k] = make_float2(a.conv_w[(size_t)cl * 4 + k], a.conv_w[(size_t)(cl + 1) * 4 + k]);
+    const float2 bias = make_float2(a.conv_b[cl], a.conv_b[cl + 1]);
     // where this channel pair goes: x, B or C (a pair never straddles two of them)
     const int gns = a.G * a.Ns;
     __nv_bfloat16 *dst;
@@ -121,22 +122,21 @@ __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
     } else {
         dst = static_cast<__nv_bfloat16 *>(a.C), width = gns, cofs = cl - a.d_inner - gns;
     }
-    dst += (size_t)b * a.N * width + cofs;
+    uint32_t *out = reinterpret_cast<uint32_t *>(dst + (size_t)b * a.N * width + cofs);
+    const int wpairs = width >> 1;  // bf16 pairs per token row of the destination
     // every input row unpacked once; the two channels' taps as packed fp32 pairs
     float2 xin[kWarpPos + kHalo];
 #pragma unroll
     for (int i = 0; i < kWarpPos + kHalo; ++i) xin[i] = tc::unpack_bf16(in[i]);
-    const float2 tap[4] = {make_float2(w0[0], w1[0]), make_float2(w0[1], w1[1]), make_float2(w0[2], w1[2]),
-                           make_float2(w0[3], w1[3])};
 #pragma unroll
     for (int j = 0; j < kWarpPos; ++j) {
         // output position s0 + j: inputs at rows j .. j + 3
-        float2 v = make_float2(b0, b1);
+        float2 v = bias;
 #pragma unroll
         for (int k = 0; k < 4; ++k) v = tc::fma_f32x2(tap[k], xin[j + k], v);
-        const int g = __shfl_sync(0xffffffffu, (j + kHalo) < 32 ? off_lo : off_hi, (j + kHalo) & 31);
-        if (g >= 0 && live)
-            *reinterpret_cast<__nv_bfloat162 *>(dst + g * width) = __floats2bfloat162_rn(silu(v.x), silu(v.y));
+        const float2 y = silu2(v);
+        const int g = __shfl_sync(0xffffffffu, g_own, j + kHalo);
+        if (g >= 0 && live) out[g * wpairs] = tc::pack_bf16(y.x, y.y);
     }
 }
 
