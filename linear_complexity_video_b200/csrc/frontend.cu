@@ -124,16 +124,18 @@ __global__ void __launch_bounds__(kThreads) front_conv_kernel(FrontArgs a)
     }
     uint32_t *out = reinterpret_cast<uint32_t *>(dst + (size_t)b * a.N * width + cofs);
     const int wpairs = width >> 1;  // bf16 pairs per token row of the destination
-    // every input row unpacked once; the two channels' taps as packed fp32 pairs
-    float2 xin[kWarpPos + kHalo];
-#pragma unroll
-    for (int i = 0; i < kWarpPos + kHalo; ++i) xin[i] = tc::unpack_bf16(in[i]);
+    // the window of rows j .. j + 3, unpacked as it slides (each row once), so that the
+    // packed rows are all the registers the loads hold
+    float2 w0 = tc::unpack_bf16(in[0]), w1 = tc::unpack_bf16(in[1]), w2 = tc::unpack_bf16(in[2]);
 #pragma unroll
     for (int j = 0; j < kWarpPos; ++j) {
         // output position s0 + j: inputs at rows j .. j + 3
-        float2 v = bias;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v = tc::fma_f32x2(tap[k], xin[j + k], v);
+        const float2 w3 = tc::unpack_bf16(in[j + kHalo]);
+        float2 v = tc::fma_f32x2(tap[0], w0, bias);
+        v = tc::fma_f32x2(tap[1], w1, v);
+        v = tc::fma_f32x2(tap[2], w2, v);
+        v = tc::fma_f32x2(tap[3], w3, v);
+        w0 = w1, w1 = w2, w2 = w3;
         const float2 y = silu2(v);
         const int g = __shfl_sync(0xffffffffu, g_own, j + kHalo);
         if (g >= 0 && live) out[g * wpairs] = tc::pack_bf16(y.x, y.y);
