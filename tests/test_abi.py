@@ -251,3 +251,27 @@ def test_gate_norm_rejects_bad_arguments():
     assert L.mate_gate_norm_fwd(y, z, w, f(1e-5), ctypes.c_void_p(base + 5120 * 2), ctypes.byref(ok), None) == \
         _lib.MATE_ERR_INVALID_ARG
     assert L.mate_gate_norm_fwd(y, z, o, f(1e-5), o, ctypes.byref(ok), None) == _lib.MATE_ERR_INVALID_ARG
+
+
+def test_python_entry_points_refuse_host_tensors():
+    """The binding has no CPU path: host tensors are refused before any library call."""
+    import torch
+    import workloads
+
+    cfg = workloads.CONFIGS["tiny"]
+    inp = workloads.generate(cfg, seed=0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mate.bissd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], 0, None, chunk=32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mate.tesa(inp["q"], inp["k"], inp["v"], cfg.Tw, cfg.Sw, cfg.shift)
+    y = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mate.gate_norm(y, y, torch.ones(64), 64)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mate.linear(y, torch.zeros(64, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mate.compose(y, y, torch.zeros(64, 64, dtype=torch.bfloat16), torch.zeros(64, 64, dtype=torch.bfloat16))
+    blk = workloads.generate_block(workloads.CONFIGS["tiny"].with_(nheads=8, headdim=16, dstate=16), d_model=64)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mate.block(blk["u"], blk, scan_mode=0, review_pool=None, chunk=32, nheads=8, headdim=16, ngroups=1,
+                   dstate=16, attn_heads=2, attn_dim=16, Tw=2, Sw=4, shift=(0, 0, 0))
