@@ -275,3 +275,42 @@ def test_python_entry_points_refuse_host_tensors():
     with pytest.raises(ValueError, match="CUDA tensor"):
         mate.block(blk["u"], blk, scan_mode=0, review_pool=None, chunk=32, nheads=8, headdim=16, ngroups=1,
                    dstate=16, attn_heads=2, attn_dim=16, Tw=2, Sw=4, shift=(0, 0, 0))
+
+
+def test_frontend_rejects_bad_arguments():
+    """mate_frontend_fwd and its workspace query check sizes, dtype, scan mode, pointers,
+    workspace and overlaps before any CUDA call."""
+    L = mate.load()
+    T, H, W = 4, 8, 8
+    ok = _lib.mate_frontend_dims(1, 256, 8, 64, 1, 64, _lib.MATE_BF16)
+    M, dc, nh = T * H * W, 8 * 64 + 2 * 64, 8
+
+    def up(n):
+        return (n + 255) // 256 * 256
+
+    assert L.mate_frontend_workspace_bytes(T, H, W, ctypes.byref(ok)) == up(M * dc * 2) + up(M * nh * 2)
+    for bad, why in [((1, 256, 6, 64, 1, 64), "heads not a multiple of 8"), ((1, 100, 8, 64, 1, 64), "d_model"),
+                     ((1, 256, 8, 64, 3, 64), "groups not dividing heads"), ((0, 256, 8, 64, 1, 64), "batch")]:
+        d = _lib.mate_frontend_dims(*bad, _lib.MATE_BF16)
+        assert L.mate_frontend_workspace_bytes(T, H, W, ctypes.byref(d)) == 0, why
+    # distinct fake device addresses, 4 GB apart (nothing is dereferenced before the checks)
+    u, w_in, cw, cb, db, z, x, dt, B, C, ws = (ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(11))
+    nbytes = L.mate_frontend_workspace_bytes(T, H, W, ctypes.byref(ok))
+
+    def call(d=ok, mode=0, **kw):
+        a = dict(u=u, w_in=w_in, cw=cw, cb=cb, db=db, z=z, x=x, dt=dt, B=B, C=C, ws=ws, n=nbytes)
+        a.update(kw)
+        return L.mate_frontend_fwd(a["u"], a["w_in"], a["cw"], a["cb"], a["db"], T, H, W, mode, a["z"], a["x"], a["dt"],
+                                   a["B"], a["C"], ctypes.byref(d) if d is not None else None, a["ws"],
+                                   ctypes.c_size_t(a["n"]), None)
+
+    assert call(d=None) == _lib.MATE_ERR_INVALID_ARG
+    assert call(mode=5) == _lib.MATE_ERR_INVALID_ARG
+    assert call(d=_lib.mate_frontend_dims(1, 256, 6, 64, 1, 64, _lib.MATE_BF16)) == _lib.MATE_ERR_UNSUPPORTED
+    assert call(d=_lib.mate_frontend_dims(1, 256, 8, 64, 1, 64, _lib.MATE_F32)) == _lib.MATE_ERR_UNSUPPORTED
+    assert call(u=None) == _lib.MATE_ERR_INVALID_ARG
+    assert call(x=ctypes.c_void_p((1 << 40) + 6 * (1 << 32) + 8)) == _lib.MATE_ERR_INVALID_ARG  # misaligned bf16
+    assert call(n=nbytes - 1) == _lib.MATE_ERR_WORKSPACE
+    assert call(ws=None) == _lib.MATE_ERR_WORKSPACE
+    assert call(x=z) == _lib.MATE_ERR_INVALID_ARG          # two outputs overlap
+    assert call(dt=u) == _lib.MATE_ERR_INVALID_ARG         # an output over an input
